@@ -1,0 +1,21 @@
+"""fp64 CPU oracle of the tensor-parallel block -- test infrastructure only.
+
+Importable only from the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline / reference leg.  The CUDA product path never touches it.
+"""
+from .tp_oracle import (  # noqa: F401
+    apply_act,
+    attn_out,
+    attn_qkv,
+    colpar_linear,
+    gelu_tanh,
+    heads_divisible,
+    linear,
+    mlp_block,
+    qkv_shard_columns,
+    rowpar_linear,
+    rowpar_partials,
+    shard_ranges,
+    shard_sum,
+    to_f64,
+)
