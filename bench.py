@@ -1,0 +1,676 @@
+#!/usr/bin/env python
+"""Benchmark of the tensor-parallel block on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sq4096|tiny|mlp70b|attn70b|mlp405b] [--tp T]
+
+Default workload: the pages' TP=2 square projection (W[4096, 4096] split by
+columns into 2 shards), decode batches T = 1, 8 and 64.  One step = one pass of
+the block's path over one batch of each T (3 column-parallel calls, 73 tokens).
+The other workloads are available for measurement with --workload.
+
+Timing: W warm-up steps, then exactly K steps captured in CUDA graphs and
+bracketed by a barrier + synchronize on both sides, timed with CUDA events on
+the launching stream; the max over ranks is taken.  Weights are rotated over
+enough copies that each step reads weights not touched for >= 4x the L2 size
+(or the weights alone exceed L2).  Multi-GPU runs are independent replicas
+(the block has no cross-GPU step here): value = all ranks' tokens / max time.
+
+--impl reference times the fp64 CPU oracle (the only reference this block
+has) on a bounded sample of the same workload on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "TP-block tokens/s; % of HBM roofline (decode) and bf16 TC peak (prefill)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["csrc/ptx.cuh", "csrc/stream_kernel.cuh", "csrc/tiled_kernel.cuh",
+                  "csrc/tp_block.cu"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    dev = device if (device is not None and dist.get_backend() == "nccl") else torch.device("cpu")
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(tokens_per_step: float, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput of `world` independent replicas timed by the slowest rank."""
+    return tokens_per_step * world / (ms_per_step_max / 1000.0)
+
+
+# ---------------------------------------------------------------- peaks, clocks, provenance
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "tensor_transformer_linear_column_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(f"{kernel}:{workload}")
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- workloads
+
+class Workload:
+    """Device-resident inputs of one workload and its step as C-ABI calls."""
+
+    def __init__(self, name: str, tp_degree, device, rotate=True):
+        import tensor_transformer_linear_column_b200 as tp
+        self.tp = tp
+        self.name = name
+        self.cfg = workloads.CONFIGS[name]
+        self.dev = device
+        cfg = self.cfg
+        if name == "sq4096":
+            self.t = tp_degree or cfg.tp_degrees[0]
+            self.Ts = list(cfg.tokens)
+            w = workloads.proj_inputs(cfg, 1)["w"]
+            self.weight_bytes = w.numel() * 2
+            self.xs = {T: workloads.normal_bf16((T, cfg.k), 1.0, 0, workloads.x_index(T))
+                       for T in self.Ts}
+            self.hidden_in, self.hidden_out = cfg.k, cfg.n
+            self.weights = [w.to(device)]
+            self.bias = None
+        elif name in ("tiny", "mlp70b", "mlp405b"):
+            self.t = tp_degree or cfg.tp_degrees[-1]
+            self.Ts = list(cfg.tokens)
+            d = workloads.mlp_inputs(cfg, self.Ts[0])
+            self.xs = {T: workloads.mlp_x(cfg, T) for T in self.Ts}
+            self.weight_bytes = (d["w1"].numel() + d["w2"].numel()) * 2
+            self.hidden_in = self.hidden_out = cfg.hidden
+            self.weights = [(d["w1"].to(device), d["w2"].to(device))]
+            self.bias = (None if d["b1"] is None else d["b1"].to(device),
+                         None if d["b2"] is None else d["b2"].to(device))
+            self.ws = torch.empty(max(tp.tp_mlp_workspace_bytes(T, cfg.ffn) for T in self.Ts),
+                                  dtype=torch.uint8, device=device)
+        elif name == "attn70b":
+            self.t = tp_degree or cfg.tp_degrees[0]
+            self.Ts = list(cfg.tokens)
+            d = workloads.attn_inputs(cfg, self.Ts[0])
+            self.xs = {self.Ts[0]: d["x"]}
+            self.ctx = d["ctx"].to(device)
+            self.weight_bytes = (d["w_qkv"].numel() + d["w_o"].numel()) * 2
+            self.hidden_in = self.hidden_out = cfg.hidden
+            self.weights = [(d["w_qkv"].to(device), d["w_o"].to(device))]
+            nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+            self.qkv = torch.empty((self.Ts[0], nqkv), dtype=torch.bfloat16, device=device)
+        else:
+            raise ValueError(name)
+        self.xd = {T: x.to(device) for T, x in self.xs.items()}
+        self.outs = {T: torch.empty((T, self.hidden_out), dtype=torch.bfloat16, device=device)
+                     for T in self.Ts}
+        # rotate weight copies so each step reads weights evicted from L2
+        self.rot = 1
+        if rotate and self.weight_bytes < 4 * L2_BYTES:
+            self.rot = int(math.ceil(4 * L2_BYTES / self.weight_bytes))
+            base = self.weights[0]
+            for _ in range(self.rot - 1):
+                if isinstance(base, tuple):
+                    self.weights.append(tuple(b.clone() for b in base))
+                else:
+                    self.weights.append(base.clone())
+        self.tokens_per_step = sum(self.Ts)
+        self.launches_per_step = len(self.Ts) * (1 if name == "sq4096" else 2)
+
+    def step(self, i: int, xs=None, outs=None):
+        tp = self.tp
+        w = self.weights[i % self.rot]
+        xs = xs or self.xd
+        outs = outs or self.outs
+        for T in self.Ts:
+            if self.name == "sq4096":
+                tp.tp_colpar_gemm_gelu(xs[T], w, None, self.t, "none", out=outs[T])
+            elif self.name == "attn70b":
+                tp.tp_attn_proj_forward(xs[T], w[0], None, self.ctx, w[1], None,
+                                        self.cfg.n_q_heads, self.cfg.n_kv_heads,
+                                        self.cfg.head_dim, self.t, qkv_out=self.qkv, out=outs[T])
+            else:
+                tp.tp_mlp_forward(xs[T], w[0], self.bias[0], w[1], self.bias[1], self.t,
+                                  self.cfg.act, out=outs[T], workspace=self.ws)
+
+    # algorithmic work of one step (for the roofline)
+    def step_bytes(self):
+        """Weights once per call + activations in and out (decode roofline)."""
+        b = 0
+        for T in self.Ts:
+            b += self.weight_bytes + 2 * T * (self.hidden_in + self.hidden_out)
+            if self.name in ("tiny", "mlp70b", "mlp405b"):
+                b += 2 * 2 * T * self.cfg.ffn  # h written and read once
+        return b
+
+    def step_flops(self):
+        f = 0
+        for T in self.Ts:
+            f += 2 * T * self.weight_bytes // 2
+        return f
+
+    def bound(self):
+        return "tensor" if max(self.Ts) > 256 else "hbm"
+
+
+class _OracleRunner:
+    _cache = {}
+
+    @classmethod
+    def get(cls, name, t):
+        key = (name, t)
+        if key not in cls._cache:
+            cls._cache[key] = cls(name, t)
+        return cls._cache[key]
+
+    def __init__(self, name, t):
+        cfg = workloads.CONFIGS[name]
+        self.name = name
+        self.cfg = cfg
+        if name == "sq4096":
+            self.t = t or cfg.tp_degrees[0]
+            self.w = workloads.proj_inputs(cfg, 1)["w"]
+            self.xs = {T: workloads.normal_bf16((T, cfg.k), 1.0, 0, workloads.x_index(T))
+                       for T in cfg.tokens}
+            self.n_out = cfg.n
+        elif name == "attn70b":
+            self.t = t or cfg.tp_degrees[0]
+            d = workloads.attn_inputs(cfg, cfg.tokens[0])
+            rows = workloads.sample_rows(cfg.tokens[0], cfg.sample_rows)
+            self.x = d["x"][rows]
+            self.ctx = d["ctx"][rows]
+            self.w_qkv, self.w_o = d["w_qkv"], d["w_o"]
+            self.n_out = cfg.hidden
+        else:
+            self.t = t or cfg.tp_degrees[-1]
+            T0 = cfg.tokens[0]
+            d = workloads.mlp_inputs(cfg, T0)
+            self.w1, self.w2, self.b1, self.b2 = d["w1"], d["w2"], d["b1"], d["b2"]
+            if cfg.sample_rows:
+                rows = workloads.sample_rows(T0, cfg.sample_rows)
+                self.xs = {T0: d["x"][rows]}
+            else:
+                self.xs = {T: workloads.mlp_x(cfg, T) for T in cfg.tokens}
+            self.n_out = cfg.hidden
+
+    def full_tokens(self):
+        """Tokens a full oracle step covers (the sampled rows for prefill workloads)."""
+        if self.name == "attn70b":
+            return self.x.shape[0]
+        return sum(x.shape[0] for x in self.xs.values())
+
+    def run(self, fraction, offset):
+        """Compute the step on output-feature block [offset, offset + fraction * n_out)."""
+        import oracle
+        n = self.n_out
+        cnt = max(64, int(round(fraction * n)) // 64 * 64)
+        j0 = (offset * cnt) % n
+        j1 = min(n, j0 + cnt)
+        if self.name == "sq4096":
+            for T, x in self.xs.items():
+                oracle.linear(x, self.w[j0:j1])
+        elif self.name == "attn70b":
+            nqkv = self.w_qkv.shape[0]
+            oracle.linear(self.x, self.w_qkv[j0 * nqkv // n:j1 * nqkv // n])
+            oracle.rowpar_linear(self.ctx, self.w_o[j0:j1], None, self.t)
+        else:
+            for T, x in self.xs.items():
+                # the first layer is needed in full for any output feature
+                h = oracle.colpar_linear(x, self.w1, self.b1, self.t, self.cfg.act) \
+                    if fraction >= 1.0 or not hasattr(self, "_h") else self._h[T]
+                if fraction < 1.0:
+                    self._h = getattr(self, "_h", {})
+                    self._h[T] = h
+                oracle.rowpar_linear(h, self.w2[j0:j1], None if self.b2 is None else self.b2[j0:j1],
+                                     self.t)
+        return (j1 - j0) / n
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def time_oracle(wl_name, t, budget_s=12.0):
+    """Oracle tokens/s on a bounded sample: whole steps while they fit the budget."""
+    runner = _OracleRunner.get(wl_name, t)
+    toks = runner.full_tokens()
+    t0 = time.perf_counter()
+    runner.run(1.0, 0)
+    one = time.perf_counter() - t0
+    steps, elapsed = 1, one
+    while elapsed + one <= budget_s:
+        t1 = time.perf_counter()
+        runner.run(1.0, 0)
+        elapsed += time.perf_counter() - t1
+        steps += 1
+    return toks * steps / elapsed, steps, elapsed, toks
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    name = args.workload
+    runner = _OracleRunner.get(name, args.tp)
+    toks = runner.full_tokens()
+    # calibrate the fraction of output features per step so the run stays short
+    t0 = time.perf_counter()
+    runner.run(1.0 / 16, 0)
+    per16 = time.perf_counter() - t0
+    total = args.steps + args.warmup
+    budget = 120.0
+    frac = min(1.0, max(1.0 / 64, (budget / max(total, 1)) / max(per16 * 16, 1e-9)))
+    for i in range(args.warmup):
+        runner.run(frac, i)
+    t0 = time.perf_counter()
+    covered = 0.0
+    for i in range(args.steps):
+        covered += runner.run(frac, i)
+    el = time.perf_counter() - t0
+    value = toks * covered / el
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle; each step covers {frac:.4f} of the output features of "
+              f"{toks} tokens ({name}); tokens/s counts full-token equivalents")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(name, runner.t, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(name, t, wl):
+    cfg = workloads.CONFIGS[name]
+    desc = {
+        "sq4096": "column-parallel projection W[4096,4096] bf16, t=2 column shards, decode T=1,8,64",
+        "tiny": "MLP block H=256 F=1024, t=2, GeLU, biases, T=8",
+        "mlp70b": "Llama-3-70B-shaped MLP decode H=8192 F=28672, GeLU, T=1,16,64",
+        "attn70b": "Llama-3-70B-shaped attention projections prefill T=4096, QKV 8192->10240 "
+                   "split by 64q/8kv heads, O-proj 8192->8192 row-split",
+        "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192",
+    }[name]
+    c = {"workload": desc, "name": name, "tp_degree": t, "tokens": list(cfg.tokens),
+         "parallelism": "replicas (per-GPU block, t logical shards on chip)"}
+    if wl is not None:
+        c["l2"] = (f"weights rotated over {wl.rot} copies "
+                   f"({wl.rot * wl.weight_bytes / 1e6:.0f} MB >= 4x the 126 MB L2)"
+                   if wl.rot > 1 else
+                   f"weights {wl.weight_bytes / 1e6:.0f} MB > 126 MB L2, read once per step")
+    return c
+
+
+def run_ours(args, world, rank, local):
+    import tensor_transformer_linear_column_b200 as tp
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    tp.load()
+    wl = Workload(args.workload, args.tp, dev, rotate=True)
+    stream = torch.cuda.Stream(device=dev)
+    K, W = args.steps, args.warmup
+
+    # graphs: one per rotation index (single step) and one of a full rotation
+    use_graph = not args.no_graph
+    g_single, g_rot = [], None
+    with torch.cuda.stream(stream):
+        for i in range(min(3, wl.rot) + 1):  # eager warm-up of each path
+            wl.step(i)
+    torch.cuda.synchronize()
+    if use_graph:
+        for i in range(wl.rot):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                wl.step(i)
+            g_single.append(g)
+        if wl.rot > 1:
+            g_rot = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rot, stream=stream):
+                for i in range(wl.rot):
+                    wl.step(i)
+
+    def run_steps(n, start=0):
+        i = start
+        if not use_graph:
+            for _ in range(n):
+                wl.step(i)
+                i += 1
+            return
+        while n > 0:
+            if g_rot is not None and i % wl.rot == 0 and n >= wl.rot:
+                g_rot.replay()
+                i += wl.rot
+                n -= wl.rot
+            else:
+                g_single[i % wl.rot].replay()
+                i += 1
+                n -= 1
+
+    with torch.cuda.stream(stream):
+        run_steps(W)
+    torch.cuda.synchronize()
+    if tp.tp_device_error_check() != tp.TP_OK:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    clk = ClockSampler(local)
+    clk.start()
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run_steps(K, start=W)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1)
+    ms_per_step = reduce_max(ms / K, world, dev)
+    value = replica_value(wl.tokens_per_step, world, ms_per_step)
+    if tp.tp_device_error_check() != tp.TP_OK:
+        raise RuntimeError("device-side timeout during the timed region")
+
+    # kernel attribution: each kernel type of the step timed alone (same inputs)
+    roof = roofline(wl, ms_per_step, stream, use_graph)
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = end_to_end(wl, stream, max(3, min(K, args.e2e_steps)), world, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, steps, el, toks = time_oracle(args.workload, args.tp, budget_s=args.cpu_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{steps} full oracle step(s) of {toks} tokens in {el:.1f} s "
+                         f"(fp64 numpy, {args.workload})"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0, sigma) bf16 inputs of the workload's shapes)",
+            "config": workload_config(args.workload, wl.t, wl),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": wl.launches_per_step * K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    del g_single, g_rot
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def roofline(wl, ms_per_step, stream, use_graph):
+    peaks, src = load_peaks()
+    if wl.bound() == "hbm":
+        # the step is nothing but the streaming kernel(s); bytes are weights +
+        # activations read once, duration = the timed region's average per step
+        achieved = wl.step_bytes() / (ms_per_step / 1000.0) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        unit = "GB/s"
+        launches = wl.launches_per_step
+        traffic = recorded_traffic("stream_gemm_kernel", wl.name)
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "stream_gemm_kernel", "launches_per_step": launches,
+                "bytes_per_step": wl.step_bytes(), "peak_source": f"{src} hbm_gbs"}
+    # tensor-bound: time each kernel of the step alone with events on the stream
+    per_kernel = kernel_durations(wl, stream)
+    name, (ms, flops) = max(per_kernel.items(), key=lambda kv: kv[1][0])
+    achieved = flops / (ms / 1000.0) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": recorded_traffic(name, wl.name),
+            "kernel": name, "kernel_ms": ms, "flops_per_launch": flops,
+            "peak_source": f"{src} bf16_tflops (burst)",
+            "per_kernel_ms": {k: v[0] for k, v in per_kernel.items()}}
+
+
+def kernel_durations(wl, stream, reps=5):
+    """Average duration of each kernel of a prefill step, timed alone with events."""
+    tp = wl.tp
+    T = wl.Ts[0]
+    out = {}
+    if wl.name == "attn70b":
+        cfg = wl.cfg
+        wq, wo = wl.weights[0]
+        nctx = cfg.n_q_heads * cfg.head_dim
+        calls = {
+            "tiled_gemm_kernel<colpar>:qkv": (
+                lambda: tp.tp_colpar_gemm_gelu(wl.xd[T], wq, None, wl.t, "none", out=wl.qkv),
+                2 * T * cfg.hidden * wq.shape[0]),
+            "tiled_gemm_kernel<rowpar>:o_proj": (
+                lambda: tp.tp_rowpar_gemm_reduce(wl.ctx, wo, None, wl.t, out=wl.outs[T]),
+                2 * T * nctx * cfg.hidden),
+        }
+    else:
+        w1, w2 = wl.weights[0]
+        F, H = wl.cfg.ffn, wl.cfg.hidden
+        h = torch.empty((T, F), dtype=torch.bfloat16, device=wl.dev)
+        calls = {
+            "tiled_gemm_kernel<colpar>:up_gelu": (
+                lambda: tp.tp_colpar_gemm_gelu(wl.xd[T], w1, wl.bias[0], wl.t, wl.cfg.act, out=h),
+                2 * T * H * F),
+            "tiled_gemm_kernel<rowpar>:down_sum": (
+                lambda: tp.tp_rowpar_gemm_reduce(h, w2, wl.bias[1], wl.t, out=wl.outs[T]),
+                2 * T * F * H),
+        }
+    for name, (fn, flops) in calls.items():
+        with torch.cuda.stream(stream):
+            fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = (e0.elapsed_time(e1) / reps, flops)
+    return out
+
+
+def end_to_end(wl, stream, steps, world, dev):
+    """Same metric through the public API with host (pinned) inputs and outputs."""
+    hx = {T: wl.xs[T].pin_memory() for T in wl.Ts}
+    hy = {T: torch.empty_like(wl.outs[T], device="cpu").pin_memory() for T in wl.Ts}
+    h2d = sum(x.numel() * 2 for x in hx.values())
+    d2h = sum(y.numel() * 2 for y in hy.values())
+    dx = {T: torch.empty_like(wl.xd[T]) for T in wl.Ts}
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            for T in wl.Ts:
+                dx[T].copy_(hx[T], non_blocking=True)
+            wl.step(i, xs=dx)
+            for T in wl.Ts:
+                hy[T].copy_(wl.outs[T], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(steps):
+            for T in wl.Ts:
+                dx[T].copy_(hx[T], non_blocking=True)
+            wl.step(i, xs=dx)
+            for T in wl.Ts:
+                hy[T].copy_(wl.outs[T], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1) / steps, world, dev)
+    barrier(world, dev)
+    return {"value": replica_value(wl.tokens_per_step, world, ms), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": steps}
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="sq4096", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--tp", type=int, default=None, help="tp degree (default: the workload's)")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
+    return args
+
+
+def main(argv=None):
+    args = parse(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

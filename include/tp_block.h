@@ -1,0 +1,196 @@
+/*
+ * tp_block.h -- C ABI of the tensor-parallel transformer block on one B200.
+ *
+ * The block is the Megatron-style split of a transformer layer (xingyuzhitong.com
+ * "Tensor vs Pipeline Parallelism", section "Tensor parallelism: split inside each
+ * layer"; drpranayjha.com "AI Infrastructure series, Part 5", section "How does
+ * tensor parallelism split a layer?"; aidolsgroup.com glossary "Tensor
+ * Parallelism", section "Full definition"):
+ *
+ *   - the first linear (MLP up-projection, or the fused QKV projection split by
+ *     heads) is split by its output features into t shards (column-parallel);
+ *   - an elementwise activation (tanh GeLU) follows on the MLP;
+ *   - the second linear (MLP down-projection, or the attention output
+ *     projection) is split by its input features into the same t shards
+ *     (row-parallel); every shard yields a full-size partial, and the partials
+ *     are summed -- the step the pages call the all-reduce.
+ *
+ * Here all t shards are logical shards on one GPU.  The all-reduce is a
+ * deterministic on-chip sum of the t partials inside the row-parallel kernel's
+ * epilogue: partial s is accumulated from zero over its own input-feature
+ * slice, the partials are added in ascending shard order in fp32, then the bias
+ * once, then one rounding to bf16.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   - Element type: bfloat16, passed as raw 16-bit patterns (tp_bf16).
+ *     Arithmetic: bf16 x bf16 products accumulated in fp32; bias, GeLU and the
+ *     shard sum in fp32; one round-to-nearest-even to bf16 on output.
+ *   - Weights are stored [out_features, in_features] row-major (the layer
+ *     computes x @ weight.T with weight shaped (out, in), iloveeagents.com
+ *     section "Example").  Activations are [tokens, features] row-major.
+ *   - Every pointer is caller-owned DEVICE memory on the current CUDA device,
+ *     16-byte aligned.  The library never allocates, frees or synchronises:
+ *     the work is enqueued asynchronously on `stream` and the call returns.
+ *     Inputs must stay valid and outputs untouched until the stream reaches
+ *     the work.  Outputs must not alias inputs.
+ *   - Sizes: T >= 1 tokens (any value); every feature dimension (K, N, H, F)
+ *     a positive multiple of 64.
+ *   - tp_degree t >= 1 must divide the dimension it splits; for the
+ *     row-parallel split the shard width (K / t) must be a multiple of 64; for
+ *     attention t must divide both head counts (xingyuzhitong.com section
+ *     "What the serving engines expose"; drpranayjha.com section "What do
+ *     people get wrong?": 64 heads split 2, 4 or 8 ways, not 3 or 6).
+ *   - Errors: argument checks run before any CUDA call; on failure the entry
+ *     point returns a tp_status != TP_OK and enqueues nothing.  A failing
+ *     CUDA call returns TP_ERR_CUDA.  No exception crosses the ABI.
+ *   - Kernels never wait without bound: a wait that runs past its limit
+ *     (about one second) records a device-side error and the kernel returns;
+ *     tp_device_error_check() reports it as TP_ERR_DEVICE_TIMEOUT.
+ *   - Results are bit-identical across repeated calls with the same
+ *     arguments, whatever the order of other work on the device.
+ *
+ * `tp_stream_t` is the same type as cudaStream_t (NULL = the legacy default
+ * stream).
+ */
+#ifndef TP_BLOCK_H_
+#define TP_BLOCK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tp_bf16;
+typedef struct CUstream_st* tp_stream_t;
+
+typedef enum tp_status {
+  TP_OK = 0,
+  TP_ERR_NULL = 1,            /* a required pointer is NULL                          */
+  TP_ERR_ALIGN = 2,           /* a pointer is not 16-byte aligned                    */
+  TP_ERR_SHAPE = 3,           /* T < 1, or a feature size not a positive multiple of 64 */
+  TP_ERR_TP_DEGREE = 4,       /* t < 1, or t does not divide what it splits          */
+  TP_ERR_WORKSPACE = 5,       /* workspace NULL or smaller than required             */
+  TP_ERR_UNSUPPORTED = 6,     /* unknown activation code or option                   */
+  TP_ERR_CUDA = 7,            /* a CUDA runtime / driver call failed                 */
+  TP_ERR_DEVICE_TIMEOUT = 8   /* a kernel's bounded wait ran out (see above)         */
+} tp_status;
+
+typedef enum tp_act {
+  TP_ACT_NONE = 0,            /* identity                                            */
+  TP_ACT_GELU_TANH = 1        /* 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))     */
+} tp_act;
+
+/*
+ * Column-parallel linear (+ bias, + activation).
+ *   out[T, N] = act(x[T, K] @ w[N, K]^T + b[N])
+ * Shard s of t owns output features [s N/t, (s+1) N/t) and computes them from
+ * the whole of x with no exchange (iloveeagents.com section "Detail", the TP=2
+ * diagram, and section "Example"); the shards' outputs side by side are `out`.
+ *   x    [T, K]  activations                    (read)
+ *   w    [N, K]  weight, output-feature major    (read)
+ *   b    [N]     bias, or NULL for none          (read)
+ *   out  [T, N]  result                          (written)
+ *   act  a tp_act value
+ * Requires N % t == 0.  Returns TP_OK or an error as described above.
+ */
+tp_status tp_colpar_gemm_gelu(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b,
+                              int T, int K, int N, int tp_degree, int act,
+                              tp_bf16* out, tp_stream_t stream);
+
+/*
+ * Row-parallel linear with the fused shard sum (the all-reduce).
+ *   P_s      = h[:, K_s] @ w[:, K_s]^T,  K_s = [s K/t, (s+1) K/t), each from zero
+ *   out[T,N] = ((P_0 + P_1) + ... + P_{t-1}) + b
+ * (xingyuzhitong.com section "Tensor parallelism: split inside each layer": the
+ * second linear layer is split by rows and the partial results are combined by
+ * an all-reduce.)
+ *   h    [T, K]  activations (the column-parallel output)  (read)
+ *   w    [N, K]  weight                                     (read)
+ *   b    [N]     bias added once after the sum, or NULL     (read)
+ *   out  [T, N]  result                                     (written)
+ * Requires K % t == 0 and (K / t) % 64 == 0.
+ */
+tp_status tp_rowpar_gemm_reduce(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b,
+                                int T, int K, int N, int tp_degree,
+                                tp_bf16* out, tp_stream_t stream);
+
+/*
+ * Bytes of workspace tp_mlp_forward needs for T tokens and FFN width F: the
+ * bf16 activation h[T, F] between the two layers, rounded up to 256 bytes.
+ * Returns 0 for T < 1 or F < 1.
+ */
+size_t tp_mlp_workspace_bytes(int T, int F);
+
+/*
+ * The tensor-parallel MLP block:
+ *   h   = act(x @ w1^T + b1)                      column-parallel, shards of F/t
+ *   out = sum_s h[:, F_s] @ w2[:, F_s]^T + b2      row-parallel, the same shards
+ * (xingyuzhitong.com section "Tensor parallelism: split inside each layer";
+ * drpranayjha.com section "How does tensor parallelism split a layer?").
+ * Column shard s of w1 feeds exactly row shard s of w2, so the activation
+ * needs no exchange; only the final partials are summed.
+ *   x  [T, H], w1 [F, H], b1 [F] or NULL, w2 [H, F], b2 [H] or NULL  (read)
+ *   out [T, H]                                                      (written)
+ *   workspace: device memory of at least tp_mlp_workspace_bytes(T, F) bytes,
+ *   16-byte aligned, holding h between the two kernels; its contents on
+ *   return are unspecified.
+ * Requires F % t == 0 and (F / t) % 64 == 0.
+ */
+tp_status tp_mlp_forward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                         const tp_bf16* w2, const tp_bf16* b2,
+                         int T, int H, int F, int tp_degree, int act,
+                         tp_bf16* out, void* workspace, size_t workspace_bytes,
+                         tp_stream_t stream);
+
+/*
+ * The attention block's two projections, split by heads.
+ *   qkv_out[T, (nq + 2 nkv) d] = x @ w_qkv^T + b_qkv     column-parallel
+ *   out[T, H] = sum_s ctx[:, G_s] @ w_o[:, G_s]^T + b_o  row-parallel
+ * Shard s owns query heads [s nq/t, (s+1) nq/t) and key-value heads
+ * [s nkv/t, (s+1) nkv/t) (attention heads distributed among the GPUs,
+ * xingyuzhitong.com section "Tensor parallelism: split inside each layer");
+ * G_s are the context columns of its query heads, (nq/t) d wide.  The
+ * attention core between the projections is not part of this library: `ctx`
+ * is the per-head context supplied by the caller.
+ *   x      [T, H]                 w_qkv [(nq + 2 nkv) d, H], columns ordered
+ *                                 Q heads | K heads | V heads, each d wide
+ *   b_qkv  [(nq + 2 nkv) d] or NULL
+ *   ctx    [T, nq d]              w_o   [H, nq d]       b_o [H] or NULL
+ *   qkv_out[T, (nq + 2 nkv) d]    out   [T, H]          (written)
+ * Requires t | nq, t | nkv, ((nq / t) d) % 64 == 0 and (nq + 2 nkv) d % 64 == 0.
+ * Key-value heads are not replicated when t > nkv: such t is rejected.
+ */
+tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_bf16* b_qkv,
+                               const tp_bf16* ctx, const tp_bf16* w_o, const tp_bf16* b_o,
+                               int T, int H, int n_q_heads, int n_kv_heads, int head_dim,
+                               int tp_degree, tp_bf16* qkv_out, tp_bf16* out,
+                               tp_stream_t stream);
+
+/* A short English description of a status code (static storage). */
+const char* tp_status_string(tp_status status);
+
+/*
+ * Synchronises the current device, then reads and clears the library's
+ * device-side error word.  Returns TP_ERR_DEVICE_TIMEOUT if any kernel of
+ * this library ran out a bounded wait since the last check, TP_ERR_CUDA if the
+ * synchronisation itself failed, TP_OK otherwise.
+ */
+tp_status tp_device_error_check(void);
+
+/*
+ * Token count at or below which a call takes the weight-streaming (decode)
+ * kernels instead of the tiled (prefill) kernels.  `max_tokens` in [0, 256];
+ * 0 sends every call to the tiled kernels.  Process-wide; returns
+ * TP_ERR_UNSUPPORTED for values outside the range.  The default is 64.
+ */
+tp_status tp_set_decode_max_tokens(int max_tokens);
+int tp_get_decode_max_tokens(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* TP_BLOCK_H_ */

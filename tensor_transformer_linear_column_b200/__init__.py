@@ -1,0 +1,214 @@
+"""Python binding of libtp_block.so (include/tp_block.h): argument marshalling only.
+
+Every function here takes torch tensors that already live on the current CUDA
+device, checks dtype / device / contiguity, and passes raw pointers, sizes and
+the current stream to the C ABI of the same name.  All arithmetic runs in the
+library's CUDA kernels; there is no fallback of any kind: if the shared library
+is missing or fails to load, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .build_lib import LIB_PATH
+
+TP_OK = 0
+TP_ERR_NULL = 1
+TP_ERR_ALIGN = 2
+TP_ERR_SHAPE = 3
+TP_ERR_TP_DEGREE = 4
+TP_ERR_WORKSPACE = 5
+TP_ERR_UNSUPPORTED = 6
+TP_ERR_CUDA = 7
+TP_ERR_DEVICE_TIMEOUT = 8
+
+TP_ACT_NONE = 0
+TP_ACT_GELU_TANH = 1
+
+ACTS = {"none": TP_ACT_NONE, "gelu_tanh": TP_ACT_GELU_TANH}
+
+# name -> (restype, argtypes) of every symbol declared in include/tp_block.h
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_Z = ctypes.c_size_t
+SIGNATURES = {
+    "tp_colpar_gemm_gelu": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "tp_rowpar_gemm_reduce": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "tp_mlp_workspace_bytes": (_Z, [_I, _I]),
+    "tp_mlp_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "tp_status_string": (ctypes.c_char_p, [_I]),
+    "tp_device_error_check": (_I, []),
+    "tp_set_decode_max_tokens": (_I, [_I]),
+    "tp_get_decode_max_tokens": (_I, []),
+}
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load the shared library (raises if it is absent: build it first)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m tensor_transformer_linear_column_b200.build_lib`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().tp_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dev: torch.device) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != TP_OK:
+        raise TPError(status, where)
+
+
+def _act(act) -> int:
+    return ACTS[act] if isinstance(act, str) else int(act)
+
+
+def tp_colpar_gemm_gelu(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor],
+                        tp_degree: int, act="none", out: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out[T, N] = act(x[T, K] @ w[N, K]^T + b) with the output split in tp_degree shards."""
+    T, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("w must be [N, K]")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    dev = x.device
+    st = load().tp_colpar_gemm_gelu(_ptr(x, "x", dev), _ptr(w, "w", dev), _ptr(b, "b", dev),
+                                    T, K, N, int(tp_degree), _act(act), _ptr(out, "out", dev),
+                                    _stream(stream))
+    _check(st, "tp_colpar_gemm_gelu")
+    return out
+
+
+def tp_rowpar_gemm_reduce(h: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor],
+                          tp_degree: int, out: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """out[T, N] = sum_s h[:, K_s] @ w[:, K_s]^T + b over tp_degree shards of K."""
+    T, K = h.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("w must be [N, K]")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=h.device)
+    dev = h.device
+    st = load().tp_rowpar_gemm_reduce(_ptr(h, "h", dev), _ptr(w, "w", dev), _ptr(b, "b", dev),
+                                      T, K, N, int(tp_degree), _ptr(out, "out", dev),
+                                      _stream(stream))
+    _check(st, "tp_rowpar_gemm_reduce")
+    return out
+
+
+def tp_mlp_workspace_bytes(T: int, F: int) -> int:
+    return int(load().tp_mlp_workspace_bytes(int(T), int(F)))
+
+
+def tp_mlp_forward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor],
+                   w2: torch.Tensor, b2: Optional[torch.Tensor], tp_degree: int,
+                   act="gelu_tanh", out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The tensor-parallel MLP block y = sum_s act(x W1_s^T + b1_s) W2[:, s]^T + b2."""
+    T, H = x.shape
+    F = w1.shape[0]
+    if w1.shape[1] != H or tuple(w2.shape) != (H, F):
+        raise ValueError("w1 must be [F, H] and w2 [H, F]")
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    need = tp_mlp_workspace_bytes(T, F)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the same device")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load().tp_mlp_forward(_ptr(x, "x", dev), _ptr(w1, "w1", dev), _ptr(b1, "b1", dev),
+                               _ptr(w2, "w2", dev), _ptr(b2, "b2", dev), T, H, F,
+                               int(tp_degree), _act(act), _ptr(out, "out", dev),
+                               workspace.data_ptr(), ws_bytes, _stream(stream))
+    _check(st, "tp_mlp_forward")
+    return out
+
+
+def tp_attn_proj_forward(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: Optional[torch.Tensor],
+                         ctx: torch.Tensor, w_o: torch.Tensor, b_o: Optional[torch.Tensor],
+                         n_q_heads: int, n_kv_heads: int, head_dim: int, tp_degree: int,
+                         qkv_out: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None):
+    """(qkv, y): the head-split QKV projection and the row-parallel output projection."""
+    T, H = x.shape
+    dev = x.device
+    nqkv = (n_q_heads + 2 * n_kv_heads) * head_dim
+    if qkv_out is None:
+        qkv_out = torch.empty((T, nqkv), dtype=torch.bfloat16, device=dev)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    st = load().tp_attn_proj_forward(_ptr(x, "x", dev), _ptr(w_qkv, "w_qkv", dev),
+                                     _ptr(b_qkv, "b_qkv", dev), _ptr(ctx, "ctx", dev),
+                                     _ptr(w_o, "w_o", dev), _ptr(b_o, "b_o", dev), T, H,
+                                     int(n_q_heads), int(n_kv_heads), int(head_dim),
+                                     int(tp_degree), _ptr(qkv_out, "qkv_out", dev),
+                                     _ptr(out, "out", dev), _stream(stream))
+    _check(st, "tp_attn_proj_forward")
+    return qkv_out, out
+
+
+def tp_device_error_check() -> int:
+    """Synchronise, then read and clear the kernels' device-side error word."""
+    return int(load().tp_device_error_check())
+
+
+def tp_set_decode_max_tokens(max_tokens: int) -> None:
+    _check(load().tp_set_decode_max_tokens(int(max_tokens)), "tp_set_decode_max_tokens")
+
+
+def tp_get_decode_max_tokens() -> int:
+    return int(load().tp_get_decode_max_tokens())

@@ -1,0 +1,347 @@
+// tp_block.cu -- the C ABI of include/tp_block.h: argument checks, path
+// choice (weight-streaming kernel for few tokens, persistent tiled kernel for
+// many), TMA descriptor encoding and kernel launches.  See the header for the
+// contract of each entry point.
+#include "tp_block.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "stream_kernel.cuh"
+#include "tiled_kernel.cuh"
+
+namespace {
+
+using tpb::StreamParams;
+using tpb::TiledParams;
+
+std::atomic<int> g_decode_max_tokens{64};
+
+constexpr int kMaxDevices = 64;
+constexpr int kStreamMaxTokens = 256;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int max_smem = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device facts and one-time kernel attributes.  Returns nullptr on failure.
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.ready) return &d;
+  int sms = 0, smem = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return nullptr;
+  if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return nullptr;
+  if (smem < tpb::kTiledSmemBytes) return nullptr;
+  if (cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           tpb::kTiledSmemBytes) != cudaSuccess)
+    return nullptr;
+  if (cudaFuncSetAttribute(tpb::tiled_gemm_kernel<true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           tpb::kTiledSmemBytes) != cudaSuccess)
+    return nullptr;
+  d.sms = sms;
+  d.max_smem = smem;
+  d.ready = true;
+  return &d;
+}
+
+// Row-major bf16 [rows, cols] viewed as 64-column x box_rows tiles with
+// 128-byte swizzling; reads outside the tensor return zeros.
+bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool feat_ok(int n) { return n > 0 && n % 64 == 0; }
+inline bool pow2_le8(int v) { return v == 1 || v == 2 || v == 4 || v == 8; }
+inline int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// ------------------------------------------------------------------ launches
+
+// Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
+// sum (1 for the column-parallel layer).  Requires T <= 256 and shards a
+// power of two <= 8 dividing K / 64.
+tp_status launch_stream(const DeviceInfo& dev, const tp_bf16* x, const tp_bf16* w,
+                        const tp_bf16* b, int T, int K, int N, int shards, int act, tp_bf16* out,
+                        cudaStream_t stream) {
+  StreamParams p{};
+  p.T = T;
+  p.K = K;
+  p.N = N;
+  p.kb_total = K / tpb::kStreamTileK;
+  p.t_pad = (T + 15) / 16 * 16;
+  p.tmem_cols = next_pow2(p.t_pad < 32 ? 32 : p.t_pad);
+  p.stage_bytes = tpb::kStreamWBytes + p.t_pad * tpb::kStreamTileK * 2;
+  int stages = (110 * 1024) / p.stage_bytes;
+  stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  p.stages = stages;
+  p.act = act;
+  p.bias = b;
+  p.out = out;
+  const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
+  const int target = 2 * dev.sms;
+  p.shards = shards;
+  const int kb_shard = p.kb_total / shards;
+  int j = 1;
+  while (shards * j * 2 <= 8 && n_tiles * shards * j < target && kb_shard / (j * 2) >= 1) j *= 2;
+  p.jsplit = j;
+  p.csize = shards * j;
+  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad);
+  if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
+
+  CUtensorMap tw, tx;
+  if (!make_tmap(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), tpb::kStreamTileM))
+    return TP_ERR_CUDA;
+  if (!make_tmap(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(K),
+                 static_cast<uint32_t>(p.t_pad)))
+    return TP_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_tiles), static_cast<unsigned>(p.csize), 1);
+  cfg.blockDim = dim3(tpb::kStreamThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(p.csize);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel, tw, tx, p) != cudaSuccess)
+    return TP_ERR_CUDA;
+  return TP_OK;
+}
+
+// Persistent tiled kernel.  segs = t accumulation segments in row-parallel
+// mode (each from zero, summed in the epilogue), 1 otherwise.
+tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
+                       const tp_bf16* b, int M, int K, int N, int segs, int act, tp_bf16* out,
+                       cudaStream_t stream) {
+  TiledParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.kb_total = K / tpb::kTiledBK;
+  p.segs = segs;
+  p.m_tiles = (M + tpb::kTiledBM - 1) / tpb::kTiledBM;
+  p.n_tiles = (N + tpb::kTiledBN - 1) / tpb::kTiledBN;
+  p.tiles = p.m_tiles * p.n_tiles;
+  p.group_m = p.m_tiles < 16 ? p.m_tiles : 16;
+  p.act = act;
+  p.bias = b;
+  p.out = out;
+
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a, static_cast<uint64_t>(M), static_cast<uint64_t>(K), tpb::kTiledBM))
+    return TP_ERR_CUDA;
+  if (!make_tmap(&tb, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), tpb::kTiledBN))
+    return TP_ERR_CUDA;
+
+  const int grid = p.tiles < dev.sms ? p.tiles : dev.sms;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(tpb::kTiledThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(tpb::kTiledSmemBytes);
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  cudaError_t e;
+  if (segs > 1)
+    e = cudaLaunchKernelEx(&cfg, tpb::tiled_gemm_kernel<true>, ta, tb, p);
+  else
+    e = cudaLaunchKernelEx(&cfg, tpb::tiled_gemm_kernel<false>, ta, tb, p);
+  return e == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status run_colpar(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T, int K, int N,
+                     int act, tp_bf16* out, cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens)
+    return launch_stream(*dev, x, w, b, T, K, N, 1, act, out, stream);
+  return launch_tiled(*dev, x, w, b, T, K, N, 1, act, out, stream);
+}
+
+tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T, int K, int N,
+                     int t, tp_bf16* out, cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens &&
+      pow2_le8(t))
+    return launch_stream(*dev, h, w, b, T, K, N, t, 0, out, stream);
+  return launch_tiled(*dev, h, w, b, T, K, N, t, 0, out, stream);
+}
+
+// ------------------------------------------------------------------ checks
+
+tp_status check_linear(const void* x, const void* w, const void* b, const void* out, int T, int K,
+                       int N, int act) {
+  if (x == nullptr || w == nullptr || out == nullptr) return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (b != nullptr && !aligned16(b)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(K) || !feat_ok(N)) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_TANH) return TP_ERR_UNSUPPORTED;
+  return TP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tp_status tp_colpar_gemm_gelu(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T, int K,
+                              int N, int tp_degree, int act, tp_bf16* out, tp_stream_t stream) {
+  tp_status s = check_linear(x, w, b, out, T, K, N, act);
+  if (s != TP_OK) return s;
+  if (tp_degree < 1 || N % tp_degree != 0) return TP_ERR_TP_DEGREE;
+  return run_colpar(x, w, b, T, K, N, act, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_rowpar_gemm_reduce(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T, int K,
+                                int N, int tp_degree, tp_bf16* out, tp_stream_t stream) {
+  tp_status s = check_linear(h, w, b, out, T, K, N, TP_ACT_NONE);
+  if (s != TP_OK) return s;
+  if (tp_degree < 1 || K % tp_degree != 0 || (K / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  return run_rowpar(h, w, b, T, K, N, tp_degree, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tp_mlp_workspace_bytes(int T, int F) {
+  if (T < 1 || F < 1) return 0;
+  const size_t raw = static_cast<size_t>(T) * static_cast<size_t>(F) * 2u;
+  return (raw + 255u) / 256u * 256u;
+}
+
+tp_status tp_mlp_forward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                         const tp_bf16* w2, const tp_bf16* b2, int T, int H, int F, int tp_degree,
+                         int act, tp_bf16* out, void* workspace, size_t workspace_bytes,
+                         tp_stream_t stream) {
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || out == nullptr) return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(out) ||
+      (b1 != nullptr && !aligned16(b1)) || (b2 != nullptr && !aligned16(b2)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || !feat_ok(F)) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_TANH) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || F % tp_degree != 0 || (F / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  if (workspace == nullptr || workspace_bytes < tp_mlp_workspace_bytes(T, F))
+    return TP_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TP_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tp_bf16* h = static_cast<tp_bf16*>(workspace);
+  tp_status s = run_colpar(x, w1, b1, T, H, F, act, h, st);
+  if (s != TP_OK) return s;
+  return run_rowpar(h, w2, b2, T, F, H, tp_degree, out, st);
+}
+
+tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_bf16* b_qkv,
+                               const tp_bf16* ctx, const tp_bf16* w_o, const tp_bf16* b_o, int T,
+                               int H, int n_q_heads, int n_kv_heads, int head_dim, int tp_degree,
+                               tp_bf16* qkv_out, tp_bf16* out, tp_stream_t stream) {
+  if (x == nullptr || w_qkv == nullptr || ctx == nullptr || w_o == nullptr ||
+      qkv_out == nullptr || out == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(ctx) || !aligned16(w_o) ||
+      !aligned16(qkv_out) || !aligned16(out) || (b_qkv != nullptr && !aligned16(b_qkv)) ||
+      (b_o != nullptr && !aligned16(b_o)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || n_q_heads < 1 || n_kv_heads < 1 || head_dim < 1)
+    return TP_ERR_SHAPE;
+  const long long nqkv = static_cast<long long>(n_q_heads + 2 * n_kv_heads) * head_dim;
+  const long long nctx = static_cast<long long>(n_q_heads) * head_dim;
+  if (nqkv > (1ll << 30) || nqkv % 64 != 0 || nctx % 64 != 0) return TP_ERR_SHAPE;
+  if (tp_degree < 1 || n_q_heads % tp_degree != 0 || n_kv_heads % tp_degree != 0 ||
+      ((n_q_heads / tp_degree) * head_dim) % 64 != 0)
+    return TP_ERR_TP_DEGREE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tp_status s = run_colpar(x, w_qkv, b_qkv, T, H, static_cast<int>(nqkv), TP_ACT_NONE, qkv_out, st);
+  if (s != TP_OK) return s;
+  return run_rowpar(ctx, w_o, b_o, T, static_cast<int>(nctx), H, tp_degree, out, st);
+}
+
+const char* tp_status_string(tp_status status) {
+  switch (status) {
+    case TP_OK: return "ok";
+    case TP_ERR_NULL: return "a required pointer is NULL";
+    case TP_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case TP_ERR_SHAPE: return "a size is out of range (T >= 1, feature sizes positive multiples of 64)";
+    case TP_ERR_TP_DEGREE: return "tp_degree does not divide the dimension or head counts it splits";
+    case TP_ERR_WORKSPACE: return "workspace missing or too small";
+    case TP_ERR_UNSUPPORTED: return "unsupported option";
+    case TP_ERR_CUDA: return "a CUDA call failed";
+    case TP_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+  }
+  return "unknown status";
+}
+
+tp_status tp_device_error_check(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return TP_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, tpb::g_tp_device_error, sizeof(v)) != cudaSuccess)
+    return TP_ERR_CUDA;
+  if (v != 0u) {
+    const unsigned int zero = 0u;
+    if (cudaMemcpyToSymbol(tpb::g_tp_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return TP_ERR_CUDA;
+    return TP_ERR_DEVICE_TIMEOUT;
+  }
+  return TP_OK;
+}
+
+tp_status tp_set_decode_max_tokens(int max_tokens) {
+  if (max_tokens < 0 || max_tokens > kStreamMaxTokens) return TP_ERR_UNSUPPORTED;
+  g_decode_max_tokens.store(max_tokens, std::memory_order_relaxed);
+  return TP_OK;
+}
+
+int tp_get_decode_max_tokens(void) { return g_decode_max_tokens.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any CUDA call.
+
+Only invalid argument combinations are passed here (with fake, never
+dereferenced pointers); each returns its error code before the library
+touches the CUDA runtime.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import tensor_transformer_linear_column_b200 as tp
+from tensor_transformer_linear_column_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp_block.h")
+
+GOOD = 0x10000          # 16-byte aligned fake device address, never dereferenced
+ODD = 0x10008 + 1       # misaligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return tp.load()
+
+
+def _header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(tp_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def _header_enum(name):
+    text = open(HEADER).read()
+    return {k: int(v) for k, v in re.findall(rf"\b({name}[A-Z0-9_]*)\s*=\s*(\d+)", text)}
+
+
+def test_header_declares_the_four_block_calls():
+    fns = _header_functions()
+    for f in ("tp_colpar_gemm_gelu", "tp_rowpar_gemm_reduce", "tp_mlp_forward",
+              "tp_attn_proj_forward"):
+        assert f in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = _header_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", build_lib.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, flags=re.M))
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(lib, name)
+    assert set(tp.SIGNATURES) == set(declared)
+
+
+def test_status_and_act_codes_match_header():
+    st = _header_enum("TP_ERR_")
+    st.update(_header_enum("TP_OK"))
+    for k, v in st.items():
+        assert getattr(tp, k) == v
+    for k, v in _header_enum("TP_ACT_").items():
+        assert getattr(tp, k) == v
+
+
+def test_status_strings(lib):
+    for code in range(0, 9):
+        s = tp.status_string(code)
+        assert isinstance(s, str) and s and s != "unknown status"
+    assert tp.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    assert tp.tp_mlp_workspace_bytes(1, 64) == 256
+    assert tp.tp_mlp_workspace_bytes(8, 1024) == 8 * 1024 * 2
+    assert tp.tp_mlp_workspace_bytes(3, 64) == 512
+    assert tp.tp_mlp_workspace_bytes(0, 64) == 0
+    assert tp.tp_mlp_workspace_bytes(8192, 53248) == 8192 * 53248 * 2
+
+
+def _colpar(lib, x=GOOD, w=GOOD, b=None, T=8, K=256, N=1024, t=2, act=0, out=GOOD):
+    return lib.tp_colpar_gemm_gelu(x, w, b, T, K, N, t, act, out, None)
+
+
+def _rowpar(lib, h=GOOD, w=GOOD, b=None, T=8, K=1024, N=256, t=2, out=GOOD):
+    return lib.tp_rowpar_gemm_reduce(h, w, b, T, K, N, t, out, None)
+
+
+def test_colpar_rejects_bad_arguments(lib):
+    assert _colpar(lib, x=None) == tp.TP_ERR_NULL
+    assert _colpar(lib, w=None) == tp.TP_ERR_NULL
+    assert _colpar(lib, out=None) == tp.TP_ERR_NULL
+    assert _colpar(lib, x=ODD) == tp.TP_ERR_ALIGN
+    assert _colpar(lib, b=ODD) == tp.TP_ERR_ALIGN
+    assert _colpar(lib, T=0) == tp.TP_ERR_SHAPE
+    assert _colpar(lib, T=-3) == tp.TP_ERR_SHAPE
+    assert _colpar(lib, K=100) == tp.TP_ERR_SHAPE
+    assert _colpar(lib, N=1000) == tp.TP_ERR_SHAPE
+    assert _colpar(lib, act=7) == tp.TP_ERR_UNSUPPORTED
+    assert _colpar(lib, t=0) == tp.TP_ERR_TP_DEGREE
+    assert _colpar(lib, N=4096, t=3) == tp.TP_ERR_TP_DEGREE
+
+
+def test_rowpar_rejects_bad_arguments(lib):
+    assert _rowpar(lib, h=None) == tp.TP_ERR_NULL
+    assert _rowpar(lib, w=ODD) == tp.TP_ERR_ALIGN
+    assert _rowpar(lib, T=0) == tp.TP_ERR_SHAPE
+    assert _rowpar(lib, t=3) == tp.TP_ERR_TP_DEGREE          # 1024 % 3 != 0
+    assert _rowpar(lib, t=32) == tp.TP_ERR_TP_DEGREE         # shard width 32 < 64
+    assert _rowpar(lib, t=-1) == tp.TP_ERR_TP_DEGREE
+
+
+def test_mlp_rejects_bad_arguments(lib):
+    def call(ws=GOOD, ws_bytes=1 << 20, t=2, F=1024, act=1, x=GOOD):
+        return lib.tp_mlp_forward(x, GOOD, None, GOOD, None, 8, 256, F, t, act, GOOD, ws,
+                                  ws_bytes, None)
+    assert call(x=None) == tp.TP_ERR_NULL
+    assert call(ws=None) == tp.TP_ERR_WORKSPACE
+    assert call(ws_bytes=8 * 1024 * 2 - 1) == tp.TP_ERR_WORKSPACE
+    assert call(ws=ODD) == tp.TP_ERR_ALIGN
+    assert call(t=3) == tp.TP_ERR_TP_DEGREE
+    assert call(t=32) == tp.TP_ERR_TP_DEGREE
+    assert call(act=5) == tp.TP_ERR_UNSUPPORTED
+    assert call(F=1000) == tp.TP_ERR_SHAPE
+
+
+def test_attention_head_rules_from_the_pages(lib, golden):
+    g = golden["head_divisibility"]
+
+    def call(t, nq=g["n_q_heads"], nkv=g["n_kv_heads"], d=128):
+        return lib.tp_attn_proj_forward(GOOD, GOOD, None, GOOD, GOOD, None, 16, 8192, nq, nkv,
+                                        d, t, GOOD, GOOD, None)
+    for t in g["tp_degrees_that_fail"]:
+        assert call(t) == tp.TP_ERR_TP_DEGREE
+    # more shards than key-value heads would need replicated heads: rejected
+    assert call(16) == tp.TP_ERR_TP_DEGREE
+    assert call(0) == tp.TP_ERR_TP_DEGREE
+    # a head group narrower than 64 columns cannot be a shard here
+    assert call(8, nq=8, nkv=8, d=32) == tp.TP_ERR_TP_DEGREE
+    assert call(1, d=6) == tp.TP_ERR_SHAPE                   # (64 + 16) * 6 columns
+
+
+def test_decode_threshold_setting(lib):
+    prev = tp.tp_get_decode_max_tokens()
+    try:
+        assert lib.tp_set_decode_max_tokens(-1) == tp.TP_ERR_UNSUPPORTED
+        assert lib.tp_set_decode_max_tokens(257) == tp.TP_ERR_UNSUPPORTED
+        tp.tp_set_decode_max_tokens(0)
+        assert tp.tp_get_decode_max_tokens() == 0
+        tp.tp_set_decode_max_tokens(128)
+        assert tp.tp_get_decode_max_tokens() == 128
+    finally:
+        tp.tp_set_decode_max_tokens(prev)
+
+
+def test_python_binding_type_checks():
+    import torch
+    x = torch.zeros(8, 256, dtype=torch.float32)
+    w = torch.zeros(1024, 256, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        tp.tp_colpar_gemm_gelu(x, w, None, 2)

@@ -1,0 +1,301 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Acceptance (bf16 in, fp32 accumulate, bf16 out): relative L2 error <= 1e-2 and
+max |error| <= 2e-2 * max |y_ref|, on the full output, or on 64 seeded rows
+for the two prefill workloads (rows are independent, so the oracle computes
+only those rows).  Both kernel paths are exercised: the weight-streaming
+(decode) kernels and the persistent tiled (prefill) kernels, forced through
+tp_set_decode_max_tokens.
+"""
+import contextlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tensor_transformer_linear_column_b200 as tp
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-2
+MAX_ABS_FRAC = 2e-2
+
+
+def _dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def assert_parity(y_gpu, y_ref, what=""):
+    y = y_gpu.detach().to("cpu", torch.float64).numpy()
+    r = np.asarray(y_ref, dtype=np.float64)
+    assert y.shape == r.shape, (what, y.shape, r.shape)
+    assert np.isfinite(y).all(), what
+    err = y - r
+    rel = np.linalg.norm(err) / max(np.linalg.norm(r), 1e-300)
+    mx = np.abs(err).max()
+    bound = MAX_ABS_FRAC * np.abs(r).max()
+    assert rel <= REL_L2 and mx <= bound, f"{what}: rel_l2={rel:.3e} max_abs={mx:.3e} bound={bound:.3e}"
+    return rel, mx
+
+
+@contextlib.contextmanager
+def kernel_path(name):
+    prev = tp.tp_get_decode_max_tokens()
+    tp.tp_set_decode_max_tokens(256 if name == "stream" else 0)
+    try:
+        yield
+    finally:
+        tp.tp_set_decode_max_tokens(prev)
+
+
+def _no_device_error():
+    assert tp.tp_device_error_check() == tp.TP_OK
+
+
+def _cuda(t, dev):
+    return None if t is None else t.to(dev).contiguous()
+
+
+# ---------------------------------------------------------------- tiny block
+
+@pytest.mark.parametrize("path", ["stream", "tiled"])
+def test_tiny_mlp_block(path):
+    dev = _dev()
+    cfg = workloads.CONFIGS["tiny"]
+    d = workloads.mlp_inputs(cfg, 8)
+    ref = oracle.mlp_block(d["x"], d["w1"], d["b1"], d["w2"], d["b2"], 2, "gelu_tanh")
+    g = {k: _cuda(v, dev) for k, v in d.items() if k != "x_fp32"}
+    with kernel_path(path):
+        y = tp.tp_mlp_forward(g["x"], g["w1"], g["b1"], g["w2"], g["b2"], 2, "gelu_tanh")
+        h = tp.tp_colpar_gemm_gelu(g["x"], g["w1"], g["b1"], 2, "gelu_tanh")
+        y2 = tp.tp_rowpar_gemm_reduce(h, g["w2"], g["b2"], 2)
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert_parity(y, ref, f"tiny mlp {path}")
+    assert torch.equal(y, y2)
+    assert_parity(h, oracle.colpar_linear(d["x"], d["w1"], d["b1"], 2, "gelu_tanh"), "tiny colpar")
+
+
+# ---------------------------------------------------------------- square projection
+
+@pytest.fixture(scope="module")
+def sq_weights():
+    cfg = workloads.CONFIGS["sq4096"]
+    d = workloads.proj_inputs(cfg, 1)
+    return cfg, d["w"]
+
+
+@pytest.mark.parametrize("path", ["stream", "tiled"])
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_sq4096_colpar(sq_weights, T, path):
+    dev = _dev()
+    cfg, w = sq_weights
+    x = workloads.proj_inputs(cfg, T)["x"]
+    ref = oracle.colpar_linear(x, w, None, 2, "none")
+    with kernel_path(path):
+        y = tp.tp_colpar_gemm_gelu(x.to(dev), w.to(dev), None, 2, "none")
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert_parity(y, ref, f"sq4096 T={T} {path}")
+
+
+# ---------------------------------------------------------------- ragged shapes, both paths
+
+RAGGED_COL = [(1, 64, 64), (3, 576, 320), (17, 128, 1088), (63, 192, 256), (65, 64, 320),
+              (130, 320, 576), (200, 256, 1024), (257, 128, 320), (300, 64, 1088)]
+
+
+@pytest.mark.parametrize("T,K,N", RAGGED_COL)
+@pytest.mark.parametrize("act", ["none", "gelu_tanh"])
+def test_colpar_ragged(T, K, N, act):
+    dev = _dev()
+    x = workloads.random_bf16_small((T, K), 1.0, 1000 + T)
+    w = workloads.random_bf16_small((N, K), 0.05, 2000 + N)
+    b = workloads.random_bf16_small((N,), 0.1, 3000 + N)
+    ref = oracle.colpar_linear(x, w, b, 1, act)
+    for path in (["stream", "tiled"] if T <= 256 else ["tiled"]):
+        with kernel_path(path):
+            y = tp.tp_colpar_gemm_gelu(x.to(dev), w.to(dev), b.to(dev), 1, act)
+        torch.cuda.synchronize()
+        assert_parity(y, ref, f"colpar T={T} K={K} N={N} {act} {path}")
+    _no_device_error()
+
+
+RAGGED_ROW = [(1, 512, 64, 1), (5, 512, 320, 2), (33, 1024, 256, 4), (64, 512, 128, 8),
+              (129, 2048, 320, 8), (300, 512, 64, 4), (7, 576, 192, 3), (40, 1024, 256, 16),
+              (2, 4096, 128, 2)]
+
+
+@pytest.mark.parametrize("T,K,N,t", RAGGED_ROW)
+def test_rowpar_ragged(T, K, N, t):
+    dev = _dev()
+    h = workloads.random_bf16_small((T, K), 0.5, 4000 + T)
+    w = workloads.random_bf16_small((N, K), 0.05, 5000 + N)
+    b = workloads.random_bf16_small((N,), 0.1, 6000 + N)
+    ref = oracle.rowpar_linear(h, w, b, t)
+    for path in (["stream", "tiled"] if T <= 256 else ["tiled"]):
+        with kernel_path(path):
+            y = tp.tp_rowpar_gemm_reduce(h.to(dev), w.to(dev), b.to(dev), t)
+        torch.cuda.synchronize()
+        assert_parity(y, ref, f"rowpar T={T} K={K} N={N} t={t} {path}")
+    _no_device_error()
+
+
+@pytest.mark.parametrize("path", ["stream", "tiled"])
+def test_rowpar_equals_sum_of_single_shard_calls(path):
+    # the all-reduce property: the fused t-shard call matches the shards'
+    # separately computed partials summed (up to rounding of those partials)
+    dev = _dev()
+    T, K, N, t = 24, 2048, 256, 4
+    h = workloads.random_bf16_small((T, K), 0.5, 71)
+    w = workloads.random_bf16_small((N, K), 0.05, 72)
+    ks = K // t
+    with kernel_path(path):
+        y = tp.tp_rowpar_gemm_reduce(h.to(dev), w.to(dev), None, t)
+        parts = [tp.tp_rowpar_gemm_reduce(h[:, s * ks:(s + 1) * ks].contiguous().to(dev),
+                                          w[:, s * ks:(s + 1) * ks].contiguous().to(dev), None, 1)
+                 for s in range(t)]
+    torch.cuda.synchronize()
+    summed = sum(p.double() for p in parts)
+    assert_parity(y, summed.cpu().numpy(), "fused sum vs separate partials")
+    assert_parity(y, oracle.rowpar_linear(h, w, None, t), "fused sum vs oracle")
+
+
+def test_colpar_result_independent_of_tp_degree():
+    dev = _dev()
+    x = workloads.random_bf16_small((9, 512), 1.0, 81).to(dev)
+    w = workloads.random_bf16_small((1024, 512), 0.05, 82).to(dev)
+    for path in ("stream", "tiled"):
+        with kernel_path(path):
+            ys = [tp.tp_colpar_gemm_gelu(x, w, None, t, "gelu_tanh") for t in (1, 2, 4, 8, 16)]
+        torch.cuda.synchronize()
+        for y in ys[1:]:
+            assert torch.equal(y, ys[0])
+
+
+# ---------------------------------------------------------------- 70B-shaped MLP decode
+
+@pytest.fixture(scope="module")
+def mlp70b():
+    cfg = workloads.CONFIGS["mlp70b"]
+    d = workloads.mlp_inputs(cfg, 1)
+    dev = _dev()
+    return cfg, d["w1"], d["w2"], d["w1"].to(dev), d["w2"].to(dev)
+
+
+@pytest.mark.parametrize("t", [4, 8])
+@pytest.mark.parametrize("T", [1, 16, 64])
+def test_mlp70b_decode(mlp70b, T, t):
+    dev = _dev()
+    cfg, w1, w2, w1d, w2d = mlp70b
+    x = workloads.mlp_x(cfg, T)
+    ref = oracle.mlp_block(x, w1, None, w2, None, t, "gelu_tanh")
+    y = tp.tp_mlp_forward(x.to(dev), w1d, None, w2d, None, t, "gelu_tanh")
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert_parity(y, ref, f"mlp70b T={T} t={t}")
+
+
+def test_mlp70b_tp4_vs_tp8_differ_only_in_rounding(mlp70b):
+    dev = _dev()
+    cfg, w1, w2, w1d, w2d = mlp70b
+    x = workloads.mlp_x(cfg, 16).to(dev)
+    y4 = tp.tp_mlp_forward(x, w1d, None, w2d, None, 4, "gelu_tanh")
+    y8 = tp.tp_mlp_forward(x, w1d, None, w2d, None, 8, "gelu_tanh")
+    torch.cuda.synchronize()
+    assert_parity(y4, y8.double().cpu().numpy(), "t=4 vs t=8")
+
+
+# ---------------------------------------------------------------- prefill, sampled rows
+
+def test_attn70b_prefill_sampled_rows():
+    dev = _dev()
+    cfg = workloads.CONFIGS["attn70b"]
+    T = cfg.tokens[0]
+    d = workloads.attn_inputs(cfg, T)
+    rows = workloads.sample_rows(T, cfg.sample_rows)
+    q_ref = oracle.attn_qkv(d["x"][rows], d["w_qkv"], None, cfg.n_q_heads, cfg.n_kv_heads,
+                            cfg.head_dim, 8)
+    o_ref = oracle.attn_out(d["ctx"][rows], d["w_o"], None, cfg.n_q_heads, cfg.head_dim, 8)
+    qkv, y = tp.tp_attn_proj_forward(d["x"].to(dev), d["w_qkv"].to(dev), None, d["ctx"].to(dev),
+                                     d["w_o"].to(dev), None, cfg.n_q_heads, cfg.n_kv_heads,
+                                     cfg.head_dim, 8)
+    torch.cuda.synchronize()
+    _no_device_error()
+    idx = torch.tensor(rows, device=dev)
+    assert_parity(qkv[idx], q_ref, "attn70b qkv")
+    assert_parity(y[idx], o_ref, "attn70b out")
+    assert torch.isfinite(y.float()).all() and torch.isfinite(qkv.float()).all()
+
+
+def test_mlp405b_prefill_sampled_rows():
+    dev = _dev()
+    cfg = workloads.CONFIGS["mlp405b"]
+    T = cfg.tokens[0]
+    d = workloads.mlp_inputs(cfg, T)
+    rows = workloads.sample_rows(T, cfg.sample_rows)
+    ref = oracle.mlp_block(d["x"][rows], d["w1"], None, d["w2"], None, 8, "gelu_tanh")
+    y = tp.tp_mlp_forward(d["x"].to(dev), d["w1"].to(dev), None, d["w2"].to(dev), None, 8,
+                          "gelu_tanh")
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert_parity(y[torch.tensor(rows, device=dev)], ref, "mlp405b rows")
+    assert torch.isfinite(y.float()).all()
+
+
+# ---------------------------------------------------------------- determinism
+
+@pytest.mark.parametrize("path", ["stream", "tiled"])
+def test_repeat_and_launch_order_bit_identical(path):
+    dev = _dev()
+    T, H, F, t = 40, 1024, 4096, 4
+    x = workloads.random_bf16_small((T, H), 1.0, 91).to(dev)
+    w1 = workloads.random_bf16_small((F, H), 0.03, 92).to(dev)
+    w2 = workloads.random_bf16_small((H, F), 0.03, 93).to(dev)
+    b2 = workloads.random_bf16_small((H,), 0.1, 94).to(dev)
+    other_x = workloads.random_bf16_small((300, H), 1.0, 95).to(dev)
+    with kernel_path(path):
+        ref = tp.tp_mlp_forward(x, w1, None, w2, b2, t, "gelu_tanh")
+        outs = []
+        for i in range(5):
+            outs.append(tp.tp_mlp_forward(x, w1, None, w2, b2, t, "gelu_tanh"))
+        # interleave other work on a second stream, then run again
+        s2 = torch.cuda.Stream()
+        with torch.cuda.stream(s2):
+            for i in range(3):
+                tp.tp_colpar_gemm_gelu(other_x, w1, None, 4, "gelu_tanh")
+        outs.append(tp.tp_mlp_forward(x, w1, None, w2, b2, t, "gelu_tanh"))
+        with torch.cuda.stream(s2):
+            outs.append(tp.tp_mlp_forward(x, w1, None, w2, b2, t, "gelu_tanh"))
+    torch.cuda.synchronize()
+    _no_device_error()
+    for o in outs:
+        assert torch.equal(o, ref)
+
+
+# ---------------------------------------------------------------- bounds: canaries
+
+@pytest.mark.parametrize("T", [1, 3, 17, 63, 129])
+def test_outputs_write_nothing_outside_their_bounds(T):
+    dev = _dev()
+    K, N, t = 256, 320, 2
+    x = workloads.random_bf16_small((T, K), 1.0, 11).to(dev)
+    w = workloads.random_bf16_small((N, K), 0.05, 12).to(dev)
+    pad = 4096
+    for path in ("stream", "tiled"):
+        buf = torch.empty((pad + T * N + pad,), dtype=torch.bfloat16, device=dev)
+        buf.view(torch.int16).fill_(0x7FC1)  # a NaN bit pattern
+        out = buf[pad:pad + T * N].view(T, N)
+        with kernel_path(path):
+            tp.tp_colpar_gemm_gelu(x, w, None, t, "gelu_tanh", out=out)
+            h = tp.tp_rowpar_gemm_reduce(x, w[:, :K].contiguous(), None, t)
+        torch.cuda.synchronize()
+        head = buf[:pad].view(torch.int16)
+        tail = buf[pad + T * N:].view(torch.int16)
+        assert bool((head == 0x7FC1).all()) and bool((tail == 0x7FC1).all()), path
+        assert torch.isfinite(out.float()).all()
+        assert torch.isfinite(h.float()).all()
+    _no_device_error()

@@ -169,6 +169,13 @@ def mlp_inputs(cfg: MLPConfig, T: int, seed: int = 0, with_bias: Optional[bool] 
     return {"x": x, "x_fp32": x32, "w1": w1, "b1": b1, "w2": w2, "b2": b2}
 
 
+def mlp_x(cfg: MLPConfig, T: int, seed: int = 0) -> torch.Tensor:
+    """Only the activations of mlp_inputs (same draw), without the weights."""
+    if cfg.x_fp32:
+        return normal_fp32((T, cfg.hidden), 1.0, seed, IDX_X).to(torch.bfloat16)
+    return normal_bf16((T, cfg.hidden), 1.0, seed, x_index(T))
+
+
 def proj_inputs(cfg: ProjConfig, T: int, seed: int = 0, with_bias: bool = False
                 ) -> Dict[str, Optional[torch.Tensor]]:
     """x [T,K], w [N,K] (and an optional b [N]) as bf16 CPU tensors."""
