@@ -1,0 +1,68 @@
+"""Host logic of bench.py on the CPU: rank plumbing, max-over-ranks timing and
+the replica aggregation, with two gloo ranks (no GPU)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    try:
+        w, r, lr = bench.dist_env()
+        assert (w, r, lr) == (world, rank, rank)
+        bench.init_dist(world, "gloo")
+        bench.barrier(world)
+        my_ms = [2.0, 3.0][rank]          # rank 1 is the slowest
+        mx = bench.reduce_max(my_ms, world)
+        val = bench.replica_value(73, world, mx)
+        bench.barrier(world)
+        dist.destroy_process_group()
+        q.put((rank, mx, val))
+    except Exception as e:  # report instead of hanging the parent
+        q.put((rank, "error", repr(e)))
+
+
+def test_two_rank_replicas_take_the_slowest_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    res.sort()
+    for rank, mx, val in res:
+        assert mx != "error", val
+        assert mx == 3.0
+        # two replicas of 73 tokens each, timed by the slowest rank
+        assert val == pytest.approx(73 * 2 / 3e-3)
+
+
+def test_single_rank_is_identity():
+    assert bench.reduce_max(1.5, 1) == 1.5
+    assert bench.replica_value(10, 1, 2.0) == pytest.approx(5000.0)
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    args = bench.parse(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert bench.run_reference(args, world=2, rank=1) == 0
+
+
+def test_cli_rejects_short_warmup():
+    with pytest.raises(SystemExit):
+        bench.parse(["--warmup", "2"])
