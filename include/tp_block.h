@@ -169,6 +169,43 @@ tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_
                                int tp_degree, tp_bf16* qkv_out, tp_bf16* out,
                                tp_stream_t stream);
 
+/*
+ * Largest activation h[T, F] (T * F * 2 bytes) that tp_mlp_forward_noalloc can
+ * hold: 4 MiB, e.g. 64 tokens at F = 28672 or 2048 tokens at F = 1024.
+ */
+#define TP_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+/*
+ * tp_mlp_forward for callers that cannot allocate device memory.
+ *
+ * The reference pages have no counterpart of this call; it exists for the
+ * callers of this library that cannot obtain scratch memory: plugin hosts
+ * that hand a kernel library only its input and output buffers (no workspace,
+ * no allocator), processes whose device memory is wholly owned by another
+ * allocator, and latency-critical loops that must not take cudaMalloc's
+ * implicit device synchronisation.
+ *
+ * Same arguments, arithmetic and results as tp_mlp_forward, minus the
+ * workspace: h lives in one TP_NOALLOC_SCRATCH_BYTES array in the library's
+ * own device memory (a static __device__ array, held by every GPU that loads
+ * the library until the process exits).  The call allocates nothing and calls
+ * no allocating routine.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture on the device.
+ *   - Every call on a device shares the one array.  Calls that may overlap
+ *     on the GPU (different streams, or other host threads) race on it and
+ *     must be ordered by the caller.  h is fully written before it is read,
+ *     so nothing needs clearing between calls.
+ * Returns TP_ERR_WORKSPACE, before any CUDA call, if T * F * 2 exceeds
+ * TP_NOALLOC_SCRATCH_BYTES; otherwise the errors of tp_mlp_forward, and
+ * TP_ERR_CUDA if the array's address cannot be obtained.
+ */
+tp_status tp_mlp_forward_noalloc(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                                 const tp_bf16* w2, const tp_bf16* b2,
+                                 int T, int H, int F, int tp_degree, int act,
+                                 tp_bf16* out, tp_stream_t stream);
+
 /* A short English description of a status code (static storage). */
 const char* tp_status_string(tp_status status);
 

@@ -41,6 +41,7 @@ SIGNATURES = {
     "tp_mlp_workspace_bytes": (_Z, [_I, _I]),
     "tp_mlp_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "tp_status_string": (ctypes.c_char_p, [_I]),
     "tp_device_error_check": (_I, []),
     "tp_set_decode_max_tokens": (_I, [_I]),
@@ -174,6 +175,31 @@ def tp_mlp_forward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor]
                                int(tp_degree), _act(act), _ptr(out, "out", dev),
                                workspace.data_ptr(), ws_bytes, _stream(stream))
     _check(st, "tp_mlp_forward")
+    return out
+
+
+TP_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
+
+
+def tp_mlp_forward_noalloc(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor],
+                           w2: torch.Tensor, b2: Optional[torch.Tensor], tp_degree: int,
+                           act="gelu_tanh", out: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """tp_mlp_forward without a workspace, for callers that cannot allocate device
+    memory: h lives in the library's own TP_NOALLOC_SCRATCH_BYTES device array,
+    shared by every call on the device (calls that may overlap on the GPU race)."""
+    T, H = x.shape
+    F = w1.shape[0]
+    if w1.shape[1] != H or tuple(w2.shape) != (H, F):
+        raise ValueError("w1 must be [F, H] and w2 [H, F]")
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    st = load().tp_mlp_forward_noalloc(_ptr(x, "x", dev), _ptr(w1, "w1", dev),
+                                       _ptr(b1, "b1", dev), _ptr(w2, "w2", dev),
+                                       _ptr(b2, "b2", dev), T, H, F, int(tp_degree), _act(act),
+                                       _ptr(out, "out", dev), _stream(stream))
+    _check(st, "tp_mlp_forward_noalloc")
     return out
 
 

@@ -345,3 +345,51 @@ tp_status tp_set_decode_max_tokens(int max_tokens) {
 int tp_get_decode_max_tokens(void) { return g_decode_max_tokens.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free MLP call
+//
+// h for tp_mlp_forward_noalloc, in the library's own device memory.  In host
+// code this name is only a host-side stand-in for the array: the device
+// address is looked up with cudaGetSymbolAddress, once per device, and cached.
+static __device__ __align__(256) unsigned char g_tp_noalloc_scratch[TP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_tp_noalloc_scratch on the current device, or nullptr.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_tp_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" tp_status tp_mlp_forward_noalloc(const tp_bf16* x, const tp_bf16* w1,
+                                            const tp_bf16* b1, const tp_bf16* w2,
+                                            const tp_bf16* b2, int T, int H, int F,
+                                            int tp_degree, int act, tp_bf16* out,
+                                            tp_stream_t stream) {
+  // every argument check comes before the first CUDA call
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || out == nullptr) return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(out) ||
+      (b1 != nullptr && !aligned16(b1)) || (b2 != nullptr && !aligned16(b2)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || !feat_ok(F)) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_TANH) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || F % tp_degree != 0 || (F / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  const size_t need = static_cast<size_t>(T) * static_cast<size_t>(F) * 2u;
+  if (need > static_cast<size_t>(TP_NOALLOC_SCRATCH_BYTES)) return TP_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (scratch == nullptr) return TP_ERR_CUDA;
+  return tp_mlp_forward(x, w1, b1, w2, b2, T, H, F, tp_degree, act, out, scratch,
+                        static_cast<size_t>(TP_NOALLOC_SCRATCH_BYTES), stream);
+}
