@@ -226,6 +226,27 @@ tp_status tp_device_error_check(void);
 tp_status tp_set_decode_max_tokens(int max_tokens);
 int tp_get_decode_max_tokens(void);
 
+/*
+ * Launch options, process-wide, a bitwise OR of:
+ *   TP_OPT_PDL             launch with programmatic dependent launch, so a
+ *                          kernel's set-up (barriers, tensor memory, descriptor
+ *                          prefetch) overlaps the tail of the preceding kernel
+ *                          on the stream.  Activations are read and outputs
+ *                          written only after that kernel has completed.  On by
+ *                          default.
+ *   TP_OPT_STATIC_WEIGHTS  with TP_OPT_PDL: a kernel may also start reading its
+ *                          weights (w, w1, w2, w_qkv, w_o) before the preceding
+ *                          kernel on the stream has completed.  Set it only when
+ *                          no kernel that may run just before a call writes that
+ *                          call's weights -- e.g. inference with weights loaded
+ *                          once.  Off by default.
+ * Returns TP_ERR_UNSUPPORTED for unknown bits (and changes nothing).
+ */
+#define TP_OPT_PDL 1u
+#define TP_OPT_STATIC_WEIGHTS 2u
+tp_status tp_set_launch_options(unsigned int flags);
+unsigned int tp_get_launch_options(void);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -29,6 +29,9 @@ TP_ERR_DEVICE_TIMEOUT = 8
 TP_ACT_NONE = 0
 TP_ACT_GELU_TANH = 1
 
+TP_OPT_PDL = 1
+TP_OPT_STATIC_WEIGHTS = 2
+
 ACTS = {"none": TP_ACT_NONE, "gelu_tanh": TP_ACT_GELU_TANH}
 
 # name -> (restype, argtypes) of every symbol declared in include/tp_block.h
@@ -46,6 +49,8 @@ SIGNATURES = {
     "tp_device_error_check": (_I, []),
     "tp_set_decode_max_tokens": (_I, [_I]),
     "tp_get_decode_max_tokens": (_I, []),
+    "tp_set_launch_options": (_I, [ctypes.c_uint]),
+    "tp_get_launch_options": (ctypes.c_uint, []),
 }
 
 
@@ -238,3 +243,12 @@ def tp_set_decode_max_tokens(max_tokens: int) -> None:
 
 def tp_get_decode_max_tokens() -> int:
     return int(load().tp_get_decode_max_tokens())
+
+
+def tp_set_launch_options(flags: int) -> None:
+    """TP_OPT_PDL | TP_OPT_STATIC_WEIGHTS (see include/tp_block.h)."""
+    _check(load().tp_set_launch_options(int(flags)), "tp_set_launch_options")
+
+
+def tp_get_launch_options() -> int:
+    return int(load().tp_get_launch_options())

@@ -255,6 +255,15 @@ __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ PDL
 
 // Wait for the preceding grid in the stream (no-op when not launched with

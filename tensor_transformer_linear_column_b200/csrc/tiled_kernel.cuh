@@ -50,6 +50,7 @@ struct TiledParams {
   int m_tiles, n_tiles, tiles;
   int group_m;    // tiles are walked in groups of group_m row-tiles
   int act;
+  int prefetch_w;  // issue the first stages' weight (B) loads before waiting for the previous grid
   const uint16_t* bias;  // [N] or nullptr
   uint16_t* out;         // [M, N]
 };
@@ -142,8 +143,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  grid_dependency_wait();
+  // the next kernel in the stream may start its own set-up now
+  grid_launch_dependents();
 
   const int kb_seg = p.kb_total / p.segs;
 
@@ -157,18 +158,38 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       for (int s = 0; s < kTiledStages; ++s) last_phase[s] = -1;
       int it = 0;
       bool ok = true;
+      // weights (B) are read-only model parameters: with prefetch_w the first
+      // stages' weight tiles are requested before the previous grid finishes
+      int pre = 0;
+      if (p.prefetch_w && blockIdx.x < p.tiles) {
+        int m0, n0;
+        tiled_coords(blockIdx.x, p, m0, n0);
+        pre = p.kb_total < kTiledStages ? p.kb_total : kTiledStages;
+        for (int kb = 0; kb < pre; ++kb) {
+          const uint32_t sa = smem_u32(smem + kb * kTiledStageBytes);
+          mbar_arrive_expect_tx(smem_u32(&full_bar[kb]), kTiledStageBytes);
+          tma_load_2d(sa + kTiledABytes, &tmap_b, smem_u32(&full_bar[kb]), kb * kTiledBK,
+                      n0 * kTiledBN);
+          last_phase[kb] = 0;
+        }
+      }
+      grid_dependency_wait();  // activations may come from the previous grid
       for (int tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x) {
         int m, n;
         tiled_coords(tile, p, m, n);
         for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
           const int s = it % kTiledStages;
           const uint32_t ph = static_cast<uint32_t>(it / kTiledStages) & 1u;
+          const uint32_t sa = smem_u32(smem + s * kTiledStageBytes);
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          if (it < pre) {  // weight half already requested
+            tma_load_2d(sa, &tmap_a, fb, kb * kTiledBK, m * kTiledBM);
+            continue;
+          }
           if (!wait_parity(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t sa = smem_u32(smem + s * kTiledStageBytes);
-          const uint32_t fb = smem_u32(&full_bar[s]);
           mbar_arrive_expect_tx(fb, kTiledStageBytes);
           tma_load_2d(sa, &tmap_a, fb, kb * kTiledBK, m * kTiledBM);
           tma_load_2d(sa + kTiledABytes, &tmap_b, fb, kb * kTiledBK, n * kTiledBN);
@@ -226,6 +247,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     __syncwarp();
   } else {
     // ---------------- epilogue warps 2..9
+    grid_dependency_wait();  // outputs may still be read by the previous grid
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
     const int ch = (warp - 2) >> 2;           // which 128-column half of the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
@@ -307,7 +329,6 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kTiledTmemCols);
   }
-  grid_launch_dependents();
 }
 
 }  // namespace tpb

@@ -21,6 +21,7 @@ using tpb::StreamParams;
 using tpb::TiledParams;
 
 std::atomic<int> g_decode_max_tokens{64};
+std::atomic<unsigned int> g_launch_options{TP_OPT_PDL};
 
 constexpr int kMaxDevices = 64;
 constexpr int kStreamMaxTokens = 256;
@@ -99,7 +100,6 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool feat_ok(int n) { return n > 0 && n % 64 == 0; }
-inline bool pow2_le8(int v) { return v == 1 || v == 2 || v == 4 || v == 8; }
 inline int next_pow2(int v) {
   int p = 1;
   while (p < v) p <<= 1;
@@ -108,12 +108,61 @@ inline int next_pow2(int v) {
 
 // ------------------------------------------------------------------ launches
 
+// Attributes shared by every launch: programmatic dependent launch (when
+// enabled) lets a kernel's set-up overlap the tail of the previous kernel on
+// the stream; the kernels wait for that kernel before touching activations or
+// outputs.
+int launch_attrs(cudaLaunchAttribute* attr, int n) {
+  if (g_launch_options.load(std::memory_order_relaxed) & TP_OPT_PDL) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  return n;
+}
+
+inline int prefetch_weights() {
+  const unsigned int o = g_launch_options.load(std::memory_order_relaxed);
+  return ((o & TP_OPT_PDL) && (o & TP_OPT_STATIC_WEIGHTS)) ? 1 : 0;
+}
+
+struct StreamGeometry {
+  int csize = 0, jsplit = 0, spc = 0;
+};
+
+// Cluster shape of the streaming kernel for n_tiles output tiles: the largest
+// cluster (1, 2, 4 or 8 CTAs along K) that keeps the grid within two CTAs per
+// SM, so every CTA is resident from the start.  Either a shard is split over
+// jsplit CTAs or a CTA owns spc whole shards (register running sum: t_pad <= 64).
+// csize == 0 when no shape fits.
+StreamGeometry stream_geometry(int n_tiles, int kb_total, int shards, int t_pad, int sms) {
+  StreamGeometry fallback;
+  const int kbs = kb_total / shards;
+  for (int csize = 8; csize >= 1; csize >>= 1) {
+    StreamGeometry g;
+    g.csize = csize;
+    if (csize >= shards) {
+      if (csize % shards != 0) continue;
+      g.jsplit = csize / shards;
+      g.spc = 1;
+      if (kbs / g.jsplit < 1) continue;
+    } else {
+      if (shards % csize != 0 || t_pad > tpb::kStreamRunCols) continue;
+      g.jsplit = 1;
+      g.spc = shards / csize;
+    }
+    if (n_tiles * csize <= 2 * sms) return g;
+    fallback = g;
+  }
+  return fallback;
+}
+
 // Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
-// sum (1 for the column-parallel layer).  Requires T <= 256 and shards a
-// power of two <= 8 dividing K / 64.
-tp_status launch_stream(const DeviceInfo& dev, const tp_bf16* x, const tp_bf16* w,
-                        const tp_bf16* b, int T, int K, int N, int shards, int act, tp_bf16* out,
-                        cudaStream_t stream) {
+// sum (1 for the column-parallel layer).  Requires T <= 256 and a geometry
+// from stream_geometry().
+tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const tp_bf16* x,
+                        const tp_bf16* w, const tp_bf16* b, int T, int K, int N, int shards,
+                        int act, tp_bf16* out, cudaStream_t stream) {
   StreamParams p{};
   p.T = T;
   p.K = K;
@@ -122,20 +171,20 @@ tp_status launch_stream(const DeviceInfo& dev, const tp_bf16* x, const tp_bf16* 
   p.t_pad = (T + 15) / 16 * 16;
   p.tmem_cols = next_pow2(p.t_pad < 32 ? 32 : p.t_pad);
   p.stage_bytes = tpb::kStreamWBytes + p.t_pad * tpb::kStreamTileK * 2;
-  int stages = (110 * 1024) / p.stage_bytes;
-  stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  // ~72 KB of pipeline: three CTAs fit on an SM, leaving room for the next
+  // kernel's CTAs to start while this one drains
+  int stages = (72 * 1024) / p.stage_bytes;
+  stages = stages < 2 ? 2 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
   p.stages = stages;
   p.act = act;
+  p.prefetch_w = prefetch_weights();
   p.bias = b;
   p.out = out;
   const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
-  const int target = 2 * dev.sms;
   p.shards = shards;
-  const int kb_shard = p.kb_total / shards;
-  int j = 1;
-  while (shards * j * 2 <= 8 && n_tiles * shards * j < target && kb_shard / (j * 2) >= 1) j *= 2;
-  p.jsplit = j;
-  p.csize = shards * j;
+  p.csize = geo.csize;
+  p.jsplit = geo.jsplit;
+  p.spc = geo.spc;
   const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad);
   if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
 
@@ -151,13 +200,13 @@ tp_status launch_stream(const DeviceInfo& dev, const tp_bf16* x, const tp_bf16* 
   cfg.blockDim = dim3(tpb::kStreamThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = static_cast<unsigned>(p.csize);
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
   if (cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel, tw, tx, p) != cudaSuccess)
     return TP_ERR_CUDA;
   return TP_OK;
@@ -179,6 +228,7 @@ tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w
   p.tiles = p.m_tiles * p.n_tiles;
   p.group_m = p.m_tiles < 16 ? p.m_tiles : 16;
   p.act = act;
+  p.prefetch_w = prefetch_weights();
   p.bias = b;
   p.out = out;
 
@@ -194,8 +244,9 @@ tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w
   cfg.blockDim = dim3(tpb::kTiledThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(tpb::kTiledSmemBytes);
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 0));
   cudaError_t e;
   if (segs > 1)
     e = cudaLaunchKernelEx(&cfg, tpb::tiled_gemm_kernel<true>, ta, tb, p);
@@ -208,8 +259,11 @@ tp_status run_colpar(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T
                      int act, tp_bf16* out, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens)
-    return launch_stream(*dev, x, w, b, T, K, N, 1, act, out, stream);
+  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens) {
+    const int t_pad = (T + 15) / 16 * 16;
+    const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, 1, t_pad, dev->sms);
+    if (g.csize > 0) return launch_stream(*dev, g, x, w, b, T, K, N, 1, act, out, stream);
+  }
   return launch_tiled(*dev, x, w, b, T, K, N, 1, act, out, stream);
 }
 
@@ -217,9 +271,11 @@ tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T
                      int t, tp_bf16* out, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens &&
-      pow2_le8(t))
-    return launch_stream(*dev, h, w, b, T, K, N, t, 0, out, stream);
+  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens) {
+    const int t_pad = (T + 15) / 16 * 16;
+    const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, t, t_pad, dev->sms);
+    if (g.csize > 0) return launch_stream(*dev, g, h, w, b, T, K, N, t, 0, out, stream);
+  }
   return launch_tiled(*dev, h, w, b, T, K, N, t, 0, out, stream);
 }
 
@@ -343,6 +399,16 @@ tp_status tp_set_decode_max_tokens(int max_tokens) {
 }
 
 int tp_get_decode_max_tokens(void) { return g_decode_max_tokens.load(std::memory_order_relaxed); }
+
+tp_status tp_set_launch_options(unsigned int flags) {
+  if ((flags & ~(TP_OPT_PDL | TP_OPT_STATIC_WEIGHTS)) != 0u) return TP_ERR_UNSUPPORTED;
+  g_launch_options.store(flags, std::memory_order_relaxed);
+  return TP_OK;
+}
+
+unsigned int tp_get_launch_options(void) {
+  return g_launch_options.load(std::memory_order_relaxed);
+}
 
 }  // extern "C"
 

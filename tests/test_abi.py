@@ -163,3 +163,17 @@ def test_python_binding_type_checks():
     w = torch.zeros(1024, 256, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         tp.tp_colpar_gemm_gelu(x, w, None, 2)
+
+
+def test_launch_options_setting(lib):
+    prev = tp.tp_get_launch_options()
+    try:
+        assert prev & tp.TP_OPT_PDL  # on by default
+        assert lib.tp_set_launch_options(4) == tp.TP_ERR_UNSUPPORTED
+        assert tp.tp_get_launch_options() == prev
+        tp.tp_set_launch_options(tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS)
+        assert tp.tp_get_launch_options() == 3
+        tp.tp_set_launch_options(0)
+        assert tp.tp_get_launch_options() == 0
+    finally:
+        tp.tp_set_launch_options(prev)

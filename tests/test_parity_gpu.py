@@ -299,3 +299,64 @@ def test_outputs_write_nothing_outside_their_bounds(T):
         assert torch.isfinite(out.float()).all()
         assert torch.isfinite(h.float()).all()
     _no_device_error()
+
+
+# ---------------------------------------------------------------- launch options (PDL)
+
+@contextlib.contextmanager
+def launch_options(flags):
+    prev = tp.tp_get_launch_options()
+    tp.tp_set_launch_options(flags)
+    try:
+        yield
+    finally:
+        tp.tp_set_launch_options(prev)
+
+
+ALL_OPTIONS = [0, tp.TP_OPT_PDL, tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS]
+
+
+@pytest.mark.parametrize("T", [5, 64, 200])
+def test_launch_options_do_not_change_results(T):
+    dev = _dev()
+    H, F, t = 512, 2048, 4
+    x = workloads.random_bf16_small((T, H), 1.0, 301).to(dev)
+    w1 = workloads.random_bf16_small((F, H), 0.04, 302).to(dev)
+    w2 = workloads.random_bf16_small((H, F), 0.04, 303).to(dev)
+    b1 = workloads.random_bf16_small((F,), 0.05, 304).to(dev)
+    outs = []
+    for flags in ALL_OPTIONS:
+        with launch_options(flags):
+            outs.append(tp.tp_mlp_forward(x, w1, b1, w2, None, t, "gelu_tanh"))
+    torch.cuda.synchronize()
+    _no_device_error()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    ref = oracle.mlp_block(x.cpu(), w1.cpu(), b1.cpu(), w2.cpu(), None, t, "gelu_tanh")
+    assert_parity(outs[-1], ref, f"options T={T}")
+
+
+@pytest.mark.parametrize("path", ["stream", "tiled"])
+def test_dependent_chain_under_programmatic_launch(path):
+    # each call reads the previous call's output: the kernels must not read
+    # activations before the producing kernel finished, whatever the options
+    dev = _dev()
+    T, K = (16, 1024) if path == "stream" else (192, 1024)
+    w = workloads.random_bf16_small((K, K), 1.0 / 32, 401).to(dev)
+    x0 = workloads.random_bf16_small((T, K), 1.0, 402).to(dev)
+    steps = 12
+    with kernel_path(path):
+        with launch_options(0):
+            ref = x0
+            for _ in range(steps):
+                ref = tp.tp_colpar_gemm_gelu(ref, w, None, 2, "gelu_tanh")
+                torch.cuda.synchronize()
+        for flags in ALL_OPTIONS[1:]:
+            with launch_options(flags):
+                y = x0
+                bufs = [torch.empty_like(x0) for _ in range(2)]
+                for i in range(steps):
+                    y = tp.tp_colpar_gemm_gelu(y, w, None, 2, "gelu_tanh", out=bufs[i % 2])
+                torch.cuda.synchronize()
+            assert torch.equal(y, ref), flags
+    _no_device_error()
