@@ -242,6 +242,43 @@ __device__ __forceinline__ void cluster_sync_all() {
                    : "memory");
 }
 
+// Split cluster barrier: every thread of every CTA in the cluster arrives once
+// per phase and then waits for the phase; release / acquire order shared
+// memory (local and remote) writes before the arrival with reads after the wait.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16, 16-byte aligned ends) from this CTA's
+// shared memory to a cluster peer's shared memory; completion is counted in
+// bytes on the mbarrier `peer_bar` in the destination CTA.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, uint32_t local_src,
+                                                  uint32_t bytes, uint32_t peer_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(peer_dst),
+      "r"(local_src), "r"(bytes), "r"(peer_bar)
+      : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy / TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Address of the same shared-memory offset in cluster CTA `rank`.
 __device__ __forceinline__ uint32_t dsmem_map(uint32_t saddr, uint32_t rank) {
   uint32_t r;

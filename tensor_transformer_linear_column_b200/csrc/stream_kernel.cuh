@@ -18,19 +18,26 @@
 // `jsplit` consecutive CTAs (csize = t * jsplit), or a CTA owns `spc`
 // consecutive whole shards (t = csize * spc).  In the second case each shard
 // is accumulated from zero in its own TMEM region (two regions, so the MMA
-// runs on while the previous shard is drained) and the four epilogue warps fold
-// the shard partials, in ascending shard order, into an fp32 running sum held
-// in registers.  Column-parallel mode is the same kernel with one shard.
+// runs on while the previous shard is drained) and the four epilogue warps
+// fold the shard partials, in ascending shard order, into an fp32 running sum
+// held in registers.  Column-parallel mode is the same kernel with one shard.
 //
-// Each CTA writes its fp32 partial [t_pad][128] to its own shared memory.
-// After a cluster barrier, CTA r sums rows [r R, (r+1) R) (R = 128 / csize)
-// across the cluster in a fixed order through distributed shared memory
-// (16-byte loads), adds the bias, applies the activation and stores bf16.
-// Nothing intermediate goes to global memory and there are no atomics, so the
-// result is bit-identical from run to run for a given shape and t.
+// Cross-CTA sum: CTA r of the cluster owns rows [r R, (r+1) R) of the tile
+// (R = 128 / csize).  Every CTA stages its fp32 partial per owner in its idle
+// pipeline buffers and sends each owner its rows with one bulk shared-memory
+// copy (cp.async.bulk, cluster scope) whose bytes complete on an mbarrier in
+// the owner; each owner waits for exactly those bytes, sums the csize partials
+// of its rows in a fixed order from its own shared memory, adds the bias,
+// applies the activation and stores bf16.  Nothing intermediate goes to global memory and there are no
+// atomics, so the result is bit-identical from run to run for a given shape
+// and t.
 //
-// Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31)
-// and do the reduction; warp 4 issues TMA; one thread of warp 5 issues MMAs.
+// Weight traffic: a ring of 3-8 stages, deeper for CTAs that stream longer;
+// with static weights the first stages are requested before the kernel waits
+// for the preceding grid, overlapping that grid's tail.
+//
+// Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
+// push and reduce; warp 4 issues TMA; one thread of warp 5 issues MMAs.
 #pragma once
 
 #include "ptx.cuh"
@@ -51,7 +58,7 @@ struct StreamParams {
   int stages;     // smem pipeline depth (<= 8)
   int stage_bytes;
   int act;        // tp_act
-  int prefetch_w; // issue the first stages' weight loads before waiting for the previous grid
+  int prefetch_w; // weights may be read before the preceding grid completes
   const uint16_t* bias;  // [N] or nullptr
   uint16_t* out;         // [T, N]
 };
@@ -66,21 +73,33 @@ constexpr int kStreamMaxStages = 8;
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
-//   [0, stages * stage_bytes)   pipeline: per stage W tile (16 KB) then x tile (t_pad * 128 B);
-//                               reused after the main loop for the fp32 partial [t_pad][128]
-//   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final, tmem slot,
-//   abort flag
-__host__ __device__ inline int stream_partial_bytes(int t_pad) { return t_pad * kStreamTileM * 4; }
-
-__host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, int t_pad) {
-  int a = stages * stage_bytes;
-  int b = stream_partial_bytes(t_pad);
-  return a > b ? a : b;
+//   [0, stages * stage_bytes)   pipeline: per stage W tile (16 KB) then x tile (t_pad * 128 B)
+//   [.., + recv_bytes)          receive buffer [csize][T][R] fp32 (<= 128 * t_pad * 4 bytes)
+//   After the main loop the pipeline buffers hold the staging [owner][T][R] fp32 of this CTA's
+//   partial (so stages * stage_bytes >= 128 * T * 4 is required: T <= 128).
+//   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final, recv,
+//   tmem slot, abort flag
+// (no receive buffer when the cluster is a single CTA: it stores directly)
+__host__ __device__ inline int stream_recv_bytes(int t_pad, int csize) {
+  return csize > 1 ? t_pad * kStreamTileM * 4 : 0;
 }
 
-__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int t_pad) {
-  return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, t_pad) +
-         (2 * stages + 5) * 8 + 16;
+__host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, int t_pad, int csize) {
+  return stages * stage_bytes + stream_recv_bytes(t_pad, csize);
+}
+
+__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int t_pad, int csize) {
+  return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, t_pad, csize) +
+         (2 * stages + 6) * 8 + 16;
+}
+
+// Epilogue of one value: bias, activation, round to bf16, store.
+__device__ __forceinline__ void stream_store(const StreamParams& p, int tok, int n, float v,
+                                             float bias) {
+  v += bias;
+  if (p.act == 1) v = gelu_tanh_f32(v);
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  p.out[static_cast<size_t>(tok) * p.N + n] = *reinterpret_cast<uint16_t*>(&h);
 }
 
 // k-block range [lo, hi) of cluster rank `crank`; never straddles a shard.
@@ -106,20 +125,24 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int data_bytes = stream_data_bytes(p.stages, p.stage_bytes, p.t_pad);
+  float* recv = reinterpret_cast<float*>(smem + p.stages * p.stage_bytes);
+  const int data_bytes = stream_data_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize);
+  const bool multi = p.csize > 1;  // partials are summed across a cluster
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + data_bytes);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + p.stages;
   uint64_t* seg_full = bars + 2 * p.stages;       // [2]
   uint64_t* seg_empty = bars + 2 * p.stages + 2;  // [2]
   uint64_t* final_bar = bars + 2 * p.stages + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+  uint64_t* recv_bar = bars + 2 * p.stages + 5;  // bytes of the peers' partials for my rows
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x;
   const int crank = static_cast<int>(cluster_ctarank());  // == blockIdx.y
+  const int R = kStreamTileM / p.csize;                   // rows each CTA finalises
 
   int kb_lo, kb_hi;
   stream_cta_range(p, crank, kb_lo, kb_hi);
@@ -137,6 +160,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       mbar_init(smem_u32(&seg_empty[b]), 4);
     }
     mbar_init(smem_u32(final_bar), 1);
+    mbar_init(smem_u32(recv_bar), 1);
+    // expect csize partials of T x R fp32 before any peer can send (phase 1)
+    mbar_arrive_expect_tx(smem_u32(recv_bar), static_cast<uint32_t>(p.csize * p.T * R * 4));
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -148,6 +174,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  // cluster phase 1: "this CTA has started" (waited on before any remote copy)
+  if (multi) cluster_arrive_relaxed();
   // the next kernel in the stream may start its own set-up now
   grid_launch_dependents();
 
@@ -160,18 +188,19 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       prefetch_tmap(&tmap_w);
       prefetch_tmap(&tmap_x);
       const uint64_t pol_w = policy_evict_first();
+      const int w_row = n_tile * kStreamTileM;
       uint32_t issued = 0u, phases = 0u;  // per stage: a load was issued / its phase bit
       // weights are read-only model parameters: with prefetch_w the first
-      // stages' weight tiles are requested before the previous grid finishes
+      // stages' weight tiles are requested before the preceding grid finishes
       const int pre = p.prefetch_w ? (nkb < p.stages ? nkb : p.stages) : 0;
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[i]), tx_bytes);
-        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[i]), (kb_lo + i) * kStreamTileK,
-                         n_tile * kStreamTileM, pol_w);
+        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[i]), (kb_lo + i) * kStreamTileK, w_row,
+                         pol_w);
         issued |= 1u << i;
       }
-      grid_dependency_wait();  // activations may come from the previous grid
+      grid_dependency_wait();  // activations may come from the preceding grid
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
         tma_load_2d(st + kStreamWBytes, &tmap_x, smem_u32(&full_bar[i]),
@@ -184,7 +213,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         const uint32_t st = smem_u32(smem + s * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[s]), tx_bytes);
         const int kc = (kb_lo + i) * kStreamTileK;
-        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[s]), kc, n_tile * kStreamTileM, pol_w);
+        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[s]), kc, w_row, pol_w);
         tma_load_2d(st + kStreamWBytes, &tmap_x, smem_u32(&full_bar[s]), kc, 0);
         issued |= 1u << s;
         phases = (phases & ~(1u << s)) | (ph << s);
@@ -240,17 +269,22 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       }
     }
     __syncwarp();
+    if (multi) cluster_wait_acquire();  // phase 1 (this warp copies nothing)
   } else {
-    // ---------------- warps 0-3: drain TMEM, fold shards in order
+    // ---------------- warps 0-3: drain TMEM, fold shards in order, stage rows per owner
     grid_dependency_wait();
-    float* part = reinterpret_cast<float*>(smem);
     const int row = warp * 32 + lane;  // TMEM lane == weight row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    // staging (the idle pipeline buffers): [owner][tok][row % R] fp32
+    float* stage_row = reinterpret_cast<float*>(smem) + (row / R) * p.T * R + (row % R);
+    // single-CTA cluster: this thread's row is final, store it directly
+    const int n_row = n_tile * kStreamTileM + row;
+    const float bias_row = (!multi && p.bias != nullptr && n_row < p.N) ? bf16_to_f32(p.bias[n_row]) : 0.0f;
     if (p.spc == 1) {
       const bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&seg_full[0]), 0, abort_flag));
       tc_fence_after();
-      // once seg_full completed every MMA is done, so the pipeline buffers are dead
-      for (int c0 = 0; c0 < p.t_pad && c0 < p.T; c0 += 16) {
+      // once seg_full completed every MMA is done, so the pipeline buffers are free
+      for (int c0 = 0; c0 < p.T; c0 += 16) {
         uint32_t r[16];
         if (ok && nkb > 0) {
           tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0), r);
@@ -259,8 +293,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) r[j] = 0u;
         }
+        if (multi) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part[(c0 + j) * kStreamTileM + row] = __uint_as_float(r[j]);
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < p.T) stage_row[(c0 + j) * R] = __uint_as_float(r[j]);
+        } else if (n_row < p.N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < p.T) stream_store(p, c0 + j, n_row, __uint_as_float(r[j]), bias_row);
+        }
       }
     } else {
       float run[kStreamRunCols];
@@ -292,40 +333,60 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&seg_empty[region]));
       }
+      if (multi) {
 #pragma unroll
-      for (int c = 0; c < kStreamRunCols / 16; ++c) {
-        if (c * 16 < p.t_pad) {
+        for (int c = 0; c < kStreamRunCols; ++c)
+          if (c < p.T) stage_row[c * R] = ok ? run[c] : 0.0f;
+      } else if (n_row < p.N) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            part[(c * 16 + j) * kStreamTileM + row] = ok ? run[c * 16 + j] : 0.0f;
-        }
+        for (int c = 0; c < kStreamRunCols; ++c)
+          if (c < p.T) stream_store(p, c, n_row, run[c], bias_row);
       }
     }
     tc_fence_before();
+    if (multi) {
+      fence_proxy_async_smem();  // staging is read by the bulk-copy engine
+      cluster_wait_acquire();    // phase 1: every CTA of the cluster has started
+      named_barrier(1, 128);     // all four warps have staged their rows
+    }
+    if (multi && threadIdx.x == 0) {
+      // one bulk copy per owner: my rows of its range -> its receive slot [crank]
+      const uint32_t bytes = static_cast<uint32_t>(p.T * R * 4);
+      for (int o = 0; o < p.csize; ++o) {
+        const uint32_t src = smem_u32(smem) + static_cast<uint32_t>(o) * bytes;
+        const uint32_t dst = dsmem_map(smem_u32(recv) + static_cast<uint32_t>(crank) * bytes,
+                                       static_cast<uint32_t>(o));
+        bulk_copy_to_peer(dst, src, bytes, dsmem_map(smem_u32(recv_bar), static_cast<uint32_t>(o)));
+      }
+    }
   }
+  if (multi && warp == kStreamProducerWarp) cluster_wait_acquire();  // phase 1 (copies nothing)
 
   __syncthreads();
   if (warp == kStreamMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_d, tcols_alloc);
   }
+  if (!multi) return;
+  if (warp >= 4) cluster_arrive_release();  // phase 2 for the warps that receive nothing
 
-  // ---------------- cluster reduction of the partials, fixed order
-  cluster_sync_all();
+  // ---------------- owner: fixed-order sum of the csize partials of its rows
   if (warp < 4) {
-    const int R = kStreamTileM / p.csize;  // rows this CTA finalises (multiple of 16)
-    const int row0 = crank * R;
+    // every peer always issues its copy, so this completes within microseconds
+    if (!drain_wait(smem_u32(recv_bar), 0, 50ull * 1000ull * 1000ull))
+      atomicOr(&g_tp_device_error, kErrTimeout);
+    // phase 2: my incoming copies have landed (so the peers' sources were read)
+    cluster_arrive_release();
     const int groups4 = R / 4;
     const int total = groups4 * p.T;
-    const uint32_t part_base = smem_u32(smem);
     for (int e = threadIdx.x; e < total; e += 128) {
       const int tok = e / groups4;
-      const int rr = row0 + (e % groups4) * 4;
-      const uint32_t off = part_base + static_cast<uint32_t>((tok * kStreamTileM + rr) * 4);
+      const int q4 = (e % groups4) * 4;
       float4 v[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        if (c < p.csize) v[c] = dsmem_ld_f32x4(dsmem_map(off, static_cast<uint32_t>(c)));
+        if (c < p.csize)
+          v[c] = *reinterpret_cast<const float4*>(recv + (c * p.T + tok) * R + q4);
       float4 y = make_float4(0.f, 0.f, 0.f, 0.f), ps = y;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -345,7 +406,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           }
         }
       }
-      const int n = n_tile * kStreamTileM + rr;
+      const int n = n_tile * kStreamTileM + crank * R + q4;
       if (n < p.N) {
         float o[4] = {y.x, y.y, y.z, y.w};
         if (p.bias != nullptr) {
@@ -364,8 +425,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       }
     }
   }
-  // peers may still be reading this CTA's partial
-  cluster_sync_all();
+  // phase 2: every CTA's incoming copies have landed, so this CTA's staging
+  // (the source of its outgoing copies) is no longer read and it may exit
+  cluster_wait_acquire();
 }
 
 }  // namespace tpb

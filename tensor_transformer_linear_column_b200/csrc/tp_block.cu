@@ -24,7 +24,7 @@ std::atomic<int> g_decode_max_tokens{64};
 std::atomic<unsigned int> g_launch_options{TP_OPT_PDL};
 
 constexpr int kMaxDevices = 64;
-constexpr int kStreamMaxTokens = 256;
+constexpr int kStreamMaxTokens = 128;
 
 struct DeviceInfo {
   bool ready = false;
@@ -86,15 +86,16 @@ const DeviceInfo* device_info() {
 // Row-major bf16 [rows, cols] viewed as 64-column x box_rows tiles with
 // 128-byte swizzling; reads outside the tensor return zeros.
 bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-               uint32_t box_rows) {
+               uint32_t box_rows, uint32_t box_cols = 64, bool swizzle = true) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -158,7 +159,7 @@ StreamGeometry stream_geometry(int n_tiles, int kb_total, int shards, int t_pad,
 }
 
 // Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
-// sum (1 for the column-parallel layer).  Requires T <= 256 and a geometry
+// sum (1 for the column-parallel layer).  Requires T <= 128 and a geometry
 // from stream_geometry().
 tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const tp_bf16* x,
                         const tp_bf16* w, const tp_bf16* b, int T, int K, int N, int shards,
@@ -171,22 +172,35 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   p.t_pad = (T + 15) / 16 * 16;
   p.tmem_cols = next_pow2(p.t_pad < 32 ? 32 : p.t_pad);
   p.stage_bytes = tpb::kStreamWBytes + p.t_pad * tpb::kStreamTileK * 2;
-  // ~72 KB of pipeline: three CTAs fit on an SM, leaving room for the next
-  // kernel's CTAs to start while this one drains
-  int stages = (72 * 1024) / p.stage_bytes;
-  stages = stages < 2 ? 2 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
-  p.stages = stages;
+  p.shards = shards;
+  p.csize = geo.csize;
+  p.jsplit = geo.jsplit;
+  p.spc = geo.spc;
+  // Ring depth: CTAs that stream >= 16 k-blocks get ~110 KB (two CTAs per SM,
+  // deep ring); short streams get ~72 KB so three CTAs fit on an SM and the
+  // next kernel's CTAs can start while this one drains.  At least 3 stages.
+  {
+    int lo, hi;
+    tpb::stream_cta_range(p, 0, lo, hi);
+    const int budget =
+        (hi - lo >= 16 ? 110 : 72) * 1024 - tpb::stream_recv_bytes(p.t_pad, p.csize);
+    int stages = budget / p.stage_bytes;
+    stages = stages < 3 ? 3 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
+    p.stages = stages;
+  }
   p.act = act;
   p.prefetch_w = prefetch_weights();
   p.bias = b;
   p.out = out;
   const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
-  p.shards = shards;
-  p.csize = geo.csize;
-  p.jsplit = geo.jsplit;
-  p.spc = geo.spc;
-  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad);
-  if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
+  // large T: the receive buffer leaves room for two stages only
+  while (p.stages > 2 &&
+         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize) > dev.max_smem)
+    --p.stages;
+  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize);
+  // the idle pipeline buffers must hold the staged partial [128][T] fp32
+  if (smem > dev.max_smem || (p.csize > 1 && p.stages * p.stage_bytes < tpb::kStreamTileM * T * 4))
+    return TP_ERR_UNSUPPORTED;
 
   CUtensorMap tw, tx;
   if (!make_tmap(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), tpb::kStreamTileM))
@@ -255,11 +269,18 @@ tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w
   return e == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
+// Weight streaming for few tokens (decode), the tiled kernel otherwise.
+bool use_stream(const DeviceInfo& dev, int T, int N) {
+  (void)dev;
+  (void)N;
+  return T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens;
+}
+
 tp_status run_colpar(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T, int K, int N,
                      int act, tp_bf16* out, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens) {
+  if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
     const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, 1, t_pad, dev->sms);
     if (g.csize > 0) return launch_stream(*dev, g, x, w, b, T, K, N, 1, act, out, stream);
@@ -271,7 +292,7 @@ tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T
                      int t, tp_bf16* out, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  if (T <= g_decode_max_tokens.load(std::memory_order_relaxed) && T <= kStreamMaxTokens) {
+  if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
     const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, t, t_pad, dev->sms);
     if (g.csize > 0) return launch_stream(*dev, g, h, w, b, T, K, N, t, 0, out, stream);

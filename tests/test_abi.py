@@ -148,7 +148,7 @@ def test_decode_threshold_setting(lib):
     prev = tp.tp_get_decode_max_tokens()
     try:
         assert lib.tp_set_decode_max_tokens(-1) == tp.TP_ERR_UNSUPPORTED
-        assert lib.tp_set_decode_max_tokens(257) == tp.TP_ERR_UNSUPPORTED
+        assert lib.tp_set_decode_max_tokens(129) == tp.TP_ERR_UNSUPPORTED
         tp.tp_set_decode_max_tokens(0)
         assert tp.tp_get_decode_max_tokens() == 0
         tp.tp_set_decode_max_tokens(128)

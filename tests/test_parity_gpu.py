@@ -43,12 +43,19 @@ def assert_parity(y_gpu, y_ref, what=""):
 
 @contextlib.contextmanager
 def kernel_path(name):
+    """Force one kernel: "stream" (tensor-core weight streaming, T <= 128) or
+    "tiled" (persistent tensor-core GEMM)."""
     prev = tp.tp_get_decode_max_tokens()
-    tp.tp_set_decode_max_tokens(256 if name == "stream" else 0)
+    tp.tp_set_decode_max_tokens(0 if name == "tiled" else 128)
     try:
         yield
     finally:
         tp.tp_set_decode_max_tokens(prev)
+
+
+def paths_for(T, K, shard_k=None):
+    """Kernels that can serve a call of T tokens."""
+    return ["stream", "tiled"] if T <= 128 else ["tiled"]
 
 
 def _no_device_error():
@@ -104,8 +111,10 @@ def test_sq4096_colpar(sq_weights, T, path):
 
 # ---------------------------------------------------------------- ragged shapes, both paths
 
-RAGGED_COL = [(1, 64, 64), (3, 576, 320), (17, 128, 1088), (63, 192, 256), (65, 64, 320),
-              (130, 320, 576), (200, 256, 1024), (257, 128, 320), (300, 64, 1088)]
+RAGGED_COL = [(1, 64, 64), (2, 768, 64), (3, 576, 320), (3, 256, 1088), (5, 4096, 320),
+              (8, 512, 64), (17, 128, 1088), (63, 192, 256), (65, 64, 320),
+              (128, 256, 384), (130, 320, 576), (200, 256, 1024), (257, 128, 320),
+              (300, 64, 1088), (5, 256, 20480), (40, 128, 20480)]
 
 
 @pytest.mark.parametrize("T,K,N", RAGGED_COL)
@@ -116,7 +125,7 @@ def test_colpar_ragged(T, K, N, act):
     w = workloads.random_bf16_small((N, K), 0.05, 2000 + N)
     b = workloads.random_bf16_small((N,), 0.1, 3000 + N)
     ref = oracle.colpar_linear(x, w, b, 1, act)
-    for path in (["stream", "tiled"] if T <= 256 else ["tiled"]):
+    for path in paths_for(T, K):
         with kernel_path(path):
             y = tp.tp_colpar_gemm_gelu(x.to(dev), w.to(dev), b.to(dev), 1, act)
         torch.cuda.synchronize()
@@ -125,8 +134,9 @@ def test_colpar_ragged(T, K, N, act):
 
 
 RAGGED_ROW = [(1, 512, 64, 1), (5, 512, 320, 2), (33, 1024, 256, 4), (64, 512, 128, 8),
-              (129, 2048, 320, 8), (300, 512, 64, 4), (7, 576, 192, 3), (40, 1024, 256, 16),
-              (2, 4096, 128, 2)]
+              (128, 1024, 192, 4), (129, 2048, 320, 8), (300, 512, 64, 4), (7, 576, 192, 3),
+              (40, 1024, 256, 16), (2, 4096, 128, 2), (3, 768, 320, 3), (6, 4096, 64, 16),
+              (8, 2048, 1088, 8), (1, 256, 64, 1)]
 
 
 @pytest.mark.parametrize("T,K,N,t", RAGGED_ROW)
@@ -136,7 +146,7 @@ def test_rowpar_ragged(T, K, N, t):
     w = workloads.random_bf16_small((N, K), 0.05, 5000 + N)
     b = workloads.random_bf16_small((N,), 0.1, 6000 + N)
     ref = oracle.rowpar_linear(h, w, b, t)
-    for path in (["stream", "tiled"] if T <= 256 else ["tiled"]):
+    for path in paths_for(T, K, K // t):
         with kernel_path(path):
             y = tp.tp_rowpar_gemm_reduce(h.to(dev), w.to(dev), b.to(dev), t)
         torch.cuda.synchronize()
@@ -166,7 +176,7 @@ def test_rowpar_equals_sum_of_single_shard_calls(path):
 
 def test_colpar_result_independent_of_tp_degree():
     dev = _dev()
-    x = workloads.random_bf16_small((9, 512), 1.0, 81).to(dev)
+    x = workloads.random_bf16_small((7, 512), 1.0, 81).to(dev)
     w = workloads.random_bf16_small((1024, 512), 0.05, 82).to(dev)
     for path in ("stream", "tiled"):
         with kernel_path(path):
@@ -285,7 +295,7 @@ def test_outputs_write_nothing_outside_their_bounds(T):
     x = workloads.random_bf16_small((T, K), 1.0, 11).to(dev)
     w = workloads.random_bf16_small((N, K), 0.05, 12).to(dev)
     pad = 4096
-    for path in ("stream", "tiled"):
+    for path in paths_for(T, K, K // t):
         buf = torch.empty((pad + T * N + pad,), dtype=torch.bfloat16, device=dev)
         buf.view(torch.int16).fill_(0x7FC1)  # a NaN bit pattern
         out = buf[pad:pad + T * N].view(T, N)
@@ -341,7 +351,7 @@ def test_dependent_chain_under_programmatic_launch(path):
     # each call reads the previous call's output: the kernels must not read
     # activations before the producing kernel finished, whatever the options
     dev = _dev()
-    T, K = (16, 1024) if path == "stream" else (192, 1024)
+    T, K = {"stream": (16, 1024), "tiled": (192, 1024)}[path]
     w = workloads.random_bf16_small((K, K), 1.0 / 32, 401).to(dev)
     x0 = workloads.random_bf16_small((T, K), 1.0, 402).to(dev)
     steps = 12
