@@ -44,8 +44,11 @@ import workloads  # noqa: E402
 METRIC = "TP-block tokens/s; % of HBM roofline (decode) and bf16 TC peak (prefill)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["csrc/ptx.cuh", "csrc/stream_kernel.cuh", "csrc/tiled_kernel.cuh",
-                  "csrc/tp_block.cu"]
+# sources whose change invalidates a kernel's recorded ncu traffic
+KERNEL_SOURCES = {
+    "stream_gemm_kernel": ["csrc/ptx.cuh", "csrc/stream_kernel.cuh", "csrc/tp_block.cu"],
+    "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/tp_block.cu"],
+}
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -102,9 +105,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel: str):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel.split("<")[0].split(":")[0]]:
         with open(os.path.join(ROOT, "tensor_transformer_linear_column_b200", rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -119,7 +122,7 @@ def recorded_traffic(kernel: str, workload: str):
         with open(p) as f:
             d = json.load(f)
         e = d.get(f"{kernel}:{workload}")
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(kernel):
             return e.get("dram_bytes_per_launch")
     except Exception:
         return None

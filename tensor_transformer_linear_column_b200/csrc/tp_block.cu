@@ -69,6 +69,11 @@ const DeviceInfo* device_info() {
   if (cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return nullptr;
+  // all of the unified L1 / shared storage as shared memory, so three ~65 KB
+  // streaming CTAs fit on an SM (the driver's default carveout allows two)
+  if (cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return nullptr;
   if (cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            tpb::kTiledSmemBytes) != cudaSuccess)
