@@ -48,6 +48,8 @@ L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = {
     "stream_gemm_kernel": ["csrc/ptx.cuh", "csrc/stream_kernel.cuh", "csrc/tp_block.cu"],
     "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/tp_block.cu"],
+    "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh",
+                         "csrc/tp_block.cu"],
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -577,7 +579,8 @@ def roofline(wl, ms_per_step, stream, use_graph, power_capped=False):
 
 
 def kernel_durations(wl, stream, reps=5):
-    """Average duration of each kernel of a prefill step, timed alone with events."""
+    """Average duration of each kernel of a prefill step, timed alone with events
+    (T > 128: both GEMMs run on the CTA-pair kernel)."""
     tp = wl.tp
     T = wl.Ts[0]
     out = {}
@@ -586,10 +589,10 @@ def kernel_durations(wl, stream, reps=5):
         wq, wo = wl.weights[0]
         nctx = cfg.n_q_heads * cfg.head_dim
         calls = {
-            "tiled_gemm_kernel<colpar>:qkv": (
+            "pair_gemm_kernel<colpar>:qkv": (
                 lambda: tp.tp_colpar_gemm_gelu(wl.xd[T], wq, None, wl.t, "none", out=wl.qkv),
                 2 * T * cfg.hidden * wq.shape[0]),
-            "tiled_gemm_kernel<rowpar>:o_proj": (
+            "pair_gemm_kernel<rowpar>:o_proj": (
                 lambda: tp.tp_rowpar_gemm_reduce(wl.ctx, wo, None, wl.t, out=wl.outs[T]),
                 2 * T * nctx * cfg.hidden),
         }
@@ -598,10 +601,10 @@ def kernel_durations(wl, stream, reps=5):
         F, H = wl.cfg.ffn, wl.cfg.hidden
         h = torch.empty((T, F), dtype=torch.bfloat16, device=wl.dev)
         calls = {
-            "tiled_gemm_kernel<colpar>:up_gelu": (
+            "pair_gemm_kernel<colpar>:up_gelu": (
                 lambda: tp.tp_colpar_gemm_gelu(wl.xd[T], w1, wl.bias[0], wl.t, wl.cfg.act, out=h),
                 2 * T * H * F),
-            "tiled_gemm_kernel<rowpar>:down_sum": (
+            "pair_gemm_kernel<rowpar>:down_sum": (
                 lambda: tp.tp_rowpar_gemm_reduce(h, w2, wl.bias[1], wl.t, out=wl.outs[T]),
                 2 * T * F * H),
         }

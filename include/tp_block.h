@@ -210,6 +210,13 @@ tp_status tp_mlp_forward_noalloc(const tp_bf16* x, const tp_bf16* w1, const tp_b
 const char* tp_status_string(tp_status status);
 
 /*
+ * Text of the last CUDA runtime / driver error that made an entry point
+ * return TP_ERR_CUDA on the calling host thread ("no CUDA error recorded"
+ * if none).  The string lives in thread-local storage until the next call.
+ */
+const char* tp_last_cuda_error(void);
+
+/*
  * Synchronises the current device, then reads and clears the library's
  * device-side error word.  Returns TP_ERR_DEVICE_TIMEOUT if any kernel of
  * this library ran out a bounded wait since the last check, TP_ERR_CUDA if the

@@ -46,6 +46,7 @@ SIGNATURES = {
     "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "tp_status_string": (ctypes.c_char_p, [_I]),
+    "tp_last_cuda_error": (ctypes.c_char_p, []),
     "tp_device_error_check": (_I, []),
     "tp_set_decode_max_tokens": (_I, [_I]),
     "tp_get_decode_max_tokens": (_I, []),
@@ -57,7 +58,10 @@ SIGNATURES = {
 class TPError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: status {status} ({status_string(status)})")
+        msg = f"{where}: status {status} ({status_string(status)})"
+        if status == TP_ERR_CUDA:
+            msg += f": {load().tp_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 _lib: Optional[ctypes.CDLL] = None

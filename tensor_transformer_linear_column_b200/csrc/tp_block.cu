@@ -9,8 +9,10 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
+#include "pair_kernel.cuh"
 #include "ptx.cuh"
 #include "stream_kernel.cuh"
 #include "tiled_kernel.cuh"
@@ -21,6 +23,16 @@ using tpb::StreamParams;
 using tpb::TiledParams;
 
 std::atomic<int> g_decode_max_tokens{64};
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+thread_local const char* g_last_cuda_call = "";
+
+// Returns true on success; otherwise remembers the error for tp_last_cuda_error().
+inline bool cuda_ok(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return true;
+  g_last_cuda_error = e;
+  g_last_cuda_call = what;
+  return false;
+}
 std::atomic<unsigned int> g_launch_options{TP_OPT_PDL};
 
 constexpr int kMaxDevices = 64;
@@ -56,31 +68,41 @@ EncodeTiledFn encode_fn() {
 // Per-device facts and one-time kernel attributes.  Returns nullptr on failure.
 const DeviceInfo* device_info() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
   if (d.ready) return &d;
   int sms = 0, smem = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+  if (!cuda_ok(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute"))
     return nullptr;
-  if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+  if (!cuda_ok(cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev),
+               "cudaDeviceGetAttribute"))
     return nullptr;
   if (smem < tpb::kTiledSmemBytes) return nullptr;
-  if (cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem), "cudaFuncSetAttribute"))
     return nullptr;
   // all of the unified L1 / shared storage as shared memory, so three ~65 KB
   // streaming CTAs fit on an SM (the driver's default carveout allows two)
-  if (cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared), "cudaFuncSetAttribute"))
     return nullptr;
-  if (cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           tpb::kTiledSmemBytes) != cudaSuccess)
+                           tpb::kTiledSmemBytes), "cudaFuncSetAttribute"))
     return nullptr;
-  if (cudaFuncSetAttribute(tpb::tiled_gemm_kernel<true>,
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::tiled_gemm_kernel<true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           tpb::kTiledSmemBytes) != cudaSuccess)
+                           tpb::kTiledSmemBytes), "cudaFuncSetAttribute"))
+    return nullptr;
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::pair_gemm_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    tpb::kPairSmemBytes),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::pair_gemm_kernel<true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    tpb::kPairSmemBytes),
+               "cudaFuncSetAttribute"))
     return nullptr;
   d.sms = sms;
   d.max_smem = smem;
@@ -93,15 +115,18 @@ const DeviceInfo* device_info() {
 bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                uint32_t box_rows, uint32_t box_cols = 64, bool swizzle = true) {
   EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
+  if (fn == nullptr) return cuda_ok(cudaErrorSymbolNotFound, "cuTensorMapEncodeTiled lookup");
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  return ok;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -226,16 +251,65 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
-  if (cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel, tw, tx, p) != cudaSuccess)
+  if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel, tw, tx, p), "launch stream_gemm_kernel"))
     return TP_ERR_CUDA;
   return TP_OK;
 }
 
+// Persistent CTA-pair kernel (256 x 256 tiles on two SMs).
+tp_status launch_pair(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
+                      const tp_bf16* b, int M, int K, int N, int segs, int act, tp_bf16* out,
+                      cudaStream_t stream) {
+  TiledParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.kb_total = K / tpb::kPairBK;
+  p.segs = segs;
+  p.m_tiles = (M + tpb::kPairBM - 1) / tpb::kPairBM;
+  p.n_tiles = (N + tpb::kPairBN - 1) / tpb::kPairBN;
+  p.tiles = p.m_tiles * p.n_tiles;
+  p.group_m = p.m_tiles < 8 ? p.m_tiles : 8;
+  p.act = act;
+  p.prefetch_w = prefetch_weights();
+  p.bias = b;
+  p.out = out;
+
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a, static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128))
+    return TP_ERR_CUDA;
+  if (!make_tmap(&tb, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), 128))
+    return TP_ERR_CUDA;
+
+  const int pairs = p.tiles < dev.sms / 2 ? p.tiles : dev.sms / 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(tpb::kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(tpb::kPairSmemBytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
+  cudaError_t e;
+  if (segs > 1)
+    e = cudaLaunchKernelEx(&cfg, tpb::pair_gemm_kernel<true>, ta, tb, p);
+  else
+    e = cudaLaunchKernelEx(&cfg, tpb::pair_gemm_kernel<false>, ta, tb, p);
+  return cuda_ok(e, "launch pair_gemm_kernel") ? TP_OK : TP_ERR_CUDA;
+}
+
 // Persistent tiled kernel.  segs = t accumulation segments in row-parallel
-// mode (each from zero, summed in the epilogue), 1 otherwise.
+// mode (each from zero, summed in the epilogue), 1 otherwise.  More than 128
+// rows go to the CTA-pair kernel.
 tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
                        const tp_bf16* b, int M, int K, int N, int segs, int act, tp_bf16* out,
                        cudaStream_t stream) {
+  if (M > tpb::kTiledBM)
+    return launch_pair(dev, a, w, b, M, K, N, segs, act, out, stream);
   TiledParams p{};
   p.M = M;
   p.N = N;
@@ -271,7 +345,7 @@ tp_status launch_tiled(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w
     e = cudaLaunchKernelEx(&cfg, tpb::tiled_gemm_kernel<true>, ta, tb, p);
   else
     e = cudaLaunchKernelEx(&cfg, tpb::tiled_gemm_kernel<false>, ta, tb, p);
-  return e == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return cuda_ok(e, "launch tiled_gemm_kernel") ? TP_OK : TP_ERR_CUDA;
 }
 
 // Weight streaming for few tokens (decode), the tiled kernel otherwise.
@@ -404,14 +478,23 @@ const char* tp_status_string(tp_status status) {
   return "unknown status";
 }
 
+const char* tp_last_cuda_error(void) {
+  static thread_local char buf[256];
+  if (g_last_cuda_error == cudaSuccess) return "no CUDA error recorded";
+  snprintf(buf, sizeof(buf), "%s: %s (%d)", g_last_cuda_call, cudaGetErrorString(g_last_cuda_error),
+           static_cast<int>(g_last_cuda_error));
+  return buf;
+}
+
 tp_status tp_device_error_check(void) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return TP_ERR_CUDA;
+  if (!cuda_ok(cudaDeviceSynchronize(), "cudaDeviceSynchronize")) return TP_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, tpb::g_tp_device_error, sizeof(v)) != cudaSuccess)
+  if (!cuda_ok(cudaMemcpyFromSymbol(&v, tpb::g_tp_device_error, sizeof(v)), "cudaMemcpyFromSymbol"))
     return TP_ERR_CUDA;
   if (v != 0u) {
     const unsigned int zero = 0u;
-    if (cudaMemcpyToSymbol(tpb::g_tp_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    if (!cuda_ok(cudaMemcpyToSymbol(tpb::g_tp_device_error, &zero, sizeof(zero)),
+                 "cudaMemcpyToSymbol"))
       return TP_ERR_CUDA;
     return TP_ERR_DEVICE_TIMEOUT;
   }
