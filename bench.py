@@ -44,12 +44,11 @@ import workloads  # noqa: E402
 METRIC = "TP-block tokens/s; % of HBM roofline (decode) and bf16 TC peak (prefill)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
-# sources whose change invalidates a kernel's recorded ncu traffic
+# device sources whose change invalidates a kernel's recorded ncu traffic
 KERNEL_SOURCES = {
-    "stream_gemm_kernel": ["csrc/ptx.cuh", "csrc/stream_kernel.cuh", "csrc/tp_block.cu"],
-    "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/tp_block.cu"],
-    "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh",
-                         "csrc/tp_block.cu"],
+    "stream_gemm_kernel": ["csrc/ptx.cuh", "csrc/stream_kernel.cuh"],
+    "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh"],
+    "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh"],
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
