@@ -12,7 +12,7 @@ The other workloads are available for measurement with --workload.
 Timing: W warm-up steps, then exactly K steps captured in CUDA graphs and
 bracketed by a barrier + synchronize on both sides, timed with CUDA events on
 the launching stream; the max over ranks is taken.  Weights are rotated over
-enough copies that each step reads weights not touched for >= 4x the L2 size
+enough copies that each call reads weights not touched for >= 4x the L2 size
 (or the weights alone exceed L2).  Multi-GPU runs are independent replicas
 (the block has no cross-GPU step here): value = all ranks' tokens / max time.
 
@@ -248,10 +248,12 @@ class Workload:
 
     def step(self, i: int, xs=None, outs=None):
         tp = self.tp
-        w = self.weights[i % self.rot]
         xs = xs or self.xd
         outs = outs or self.outs
-        for T in self.Ts:
+        for j, T in enumerate(self.Ts):
+            # every call of every step reads a weight copy not touched for
+            # rot - 1 calls, so weights come from HBM, never from L2
+            w = self.weights[(i * len(self.Ts) + j) % self.rot]
             if self.name == "sq4096":
                 tp.tp_colpar_gemm_gelu(xs[T], w, None, self.t, "none", out=outs[T])
             elif self.name == "attn70b":
@@ -433,8 +435,9 @@ def workload_config(name, t, wl):
     c = {"workload": desc, "name": name, "tp_degree": t, "tokens": list(cfg.tokens),
          "parallelism": "replicas (per-GPU block, t logical shards on chip)"}
     if wl is not None:
-        c["l2"] = (f"weights rotated over {wl.rot} copies "
-                   f"({wl.rot * wl.weight_bytes / 1e6:.0f} MB >= 4x the 126 MB L2)"
+        c["l2"] = (f"weights rotated per call over {wl.rot} copies "
+                   f"({wl.rot * wl.weight_bytes / 1e6:.0f} MB >= 4x the 126 MB L2): every call "
+                   f"reads cold weights"
                    if wl.rot > 1 else
                    f"weights {wl.weight_bytes / 1e6:.0f} MB > 126 MB L2, read once per step")
     return c

@@ -66,3 +66,17 @@ def test_reference_arm_other_ranks_do_no_work():
 def test_cli_rejects_short_warmup():
     with pytest.raises(SystemExit):
         bench.parse(["--warmup", "2"])
+
+
+def test_reference_arm_times_the_oracle_on_cpu(capsys):
+    # the reference arm of the contract: the fp64 oracle on a bounded sample
+    import json
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "3"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["metric"] == bench.METRIC

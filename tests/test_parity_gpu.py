@@ -58,6 +58,20 @@ def paths_for(T, K, shard_k=None):
     return ["stream", "tiled"] if T <= 128 else ["tiled"]
 
 
+@contextlib.contextmanager
+def launch_options(flags):
+    prev = tp.tp_get_launch_options()
+    tp.tp_set_launch_options(flags)
+    try:
+        yield
+    finally:
+        tp.tp_set_launch_options(prev)
+
+
+# the launch configuration bench.py times: PDL with static-weight prefetch
+BENCH_OPTIONS = tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS
+
+
 def _no_device_error():
     assert tp.tp_device_error_check() == tp.TP_OK
 
@@ -102,7 +116,7 @@ def test_sq4096_colpar(sq_weights, T, path):
     cfg, w = sq_weights
     x = workloads.proj_inputs(cfg, T)["x"]
     ref = oracle.colpar_linear(x, w, None, 2, "none")
-    with kernel_path(path):
+    with kernel_path(path), launch_options(BENCH_OPTIONS):
         y = tp.tp_colpar_gemm_gelu(x.to(dev), w.to(dev), None, 2, "none")
     torch.cuda.synchronize()
     _no_device_error()
@@ -203,7 +217,8 @@ def test_mlp70b_decode(mlp70b, T, t):
     cfg, w1, w2, w1d, w2d = mlp70b
     x = workloads.mlp_x(cfg, T)
     ref = oracle.mlp_block(x, w1, None, w2, None, t, "gelu_tanh")
-    y = tp.tp_mlp_forward(x.to(dev), w1d, None, w2d, None, t, "gelu_tanh")
+    with launch_options(BENCH_OPTIONS):
+        y = tp.tp_mlp_forward(x.to(dev), w1d, None, w2d, None, t, "gelu_tanh")
     torch.cuda.synchronize()
     _no_device_error()
     assert_parity(y, ref, f"mlp70b T={T} t={t}")
@@ -230,9 +245,10 @@ def test_attn70b_prefill_sampled_rows():
     q_ref = oracle.attn_qkv(d["x"][rows], d["w_qkv"], None, cfg.n_q_heads, cfg.n_kv_heads,
                             cfg.head_dim, 8)
     o_ref = oracle.attn_out(d["ctx"][rows], d["w_o"], None, cfg.n_q_heads, cfg.head_dim, 8)
-    qkv, y = tp.tp_attn_proj_forward(d["x"].to(dev), d["w_qkv"].to(dev), None, d["ctx"].to(dev),
-                                     d["w_o"].to(dev), None, cfg.n_q_heads, cfg.n_kv_heads,
-                                     cfg.head_dim, 8)
+    with launch_options(BENCH_OPTIONS):
+        qkv, y = tp.tp_attn_proj_forward(d["x"].to(dev), d["w_qkv"].to(dev), None,
+                                         d["ctx"].to(dev), d["w_o"].to(dev), None,
+                                         cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, 8)
     torch.cuda.synchronize()
     _no_device_error()
     idx = torch.tensor(rows, device=dev)
@@ -248,8 +264,9 @@ def test_mlp405b_prefill_sampled_rows():
     d = workloads.mlp_inputs(cfg, T)
     rows = workloads.sample_rows(T, cfg.sample_rows)
     ref = oracle.mlp_block(d["x"][rows], d["w1"], None, d["w2"], None, 8, "gelu_tanh")
-    y = tp.tp_mlp_forward(d["x"].to(dev), d["w1"].to(dev), None, d["w2"].to(dev), None, 8,
-                          "gelu_tanh")
+    with launch_options(BENCH_OPTIONS):
+        y = tp.tp_mlp_forward(d["x"].to(dev), d["w1"].to(dev), None, d["w2"].to(dev), None, 8,
+                              "gelu_tanh")
     torch.cuda.synchronize()
     _no_device_error()
     assert_parity(y[torch.tensor(rows, device=dev)], ref, "mlp405b rows")
@@ -313,15 +330,6 @@ def test_outputs_write_nothing_outside_their_bounds(T):
 
 # ---------------------------------------------------------------- launch options (PDL)
 
-@contextlib.contextmanager
-def launch_options(flags):
-    prev = tp.tp_get_launch_options()
-    tp.tp_set_launch_options(flags)
-    try:
-        yield
-    finally:
-        tp.tp_set_launch_options(prev)
-
 
 ALL_OPTIONS = [0, tp.TP_OPT_PDL, tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS]
 
@@ -370,3 +378,29 @@ def test_dependent_chain_under_programmatic_launch(path):
                 torch.cuda.synchronize()
             assert torch.equal(y, ref), flags
     _no_device_error()
+
+
+def test_graph_replayed_decode_step_matches_eager(sq_weights):
+    # the default bench step (T = 1, 8, 64 on the 4096 x 4096 projection, weights
+    # rotated per call) captured in a CUDA graph gives the eager results bit for bit
+    dev = _dev()
+    cfg, w = sq_weights
+    ws = [w.to(dev), (w.to(dev).float() * 0.5).to(torch.bfloat16)]
+    xs = {T: workloads.proj_inputs(cfg, T)["x"].to(dev) for T in (1, 8, 64)}
+    outs = {T: torch.empty((T, 4096), dtype=torch.bfloat16, device=dev) for T in xs}
+    with launch_options(BENCH_OPTIONS):
+        eager = {}
+        for j, T in enumerate(xs):
+            eager[T] = tp.tp_colpar_gemm_gelu(xs[T], ws[j % 2], None, 2, "none")
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for j, T in enumerate(xs):
+                tp.tp_colpar_gemm_gelu(xs[T], ws[j % 2], None, 2, "none", out=outs[T])
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    _no_device_error()
+    for T in xs:
+        assert torch.equal(outs[T], eager[T])
+    assert_parity(outs[64], oracle.colpar_linear(xs[64].cpu(), w, None, 2, "none"), "graph T=64")
