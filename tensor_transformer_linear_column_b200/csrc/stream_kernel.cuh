@@ -119,7 +119,12 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
   }
 }
 
-__global__ void __launch_bounds__(kStreamThreads, 1)
+// kShards = false: one accumulation segment per CTA (spc == 1); registers are
+// bounded so three CTAs fit on an SM (six warps are granted registers as
+// eight), which lets the next call's CTAs start and prefetch weights while
+// this call drains.  kShards = true: several shards per CTA (spc >= 1).
+template <bool kShards>
+__global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
     stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_x, const StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     // single-CTA cluster: this thread's row is final, store it directly
     const int n_row = n_tile * kStreamTileM + row;
     const float bias_row = (!multi && p.bias != nullptr && n_row < p.N) ? bf16_to_f32(p.bias[n_row]) : 0.0f;
-    if (p.spc == 1) {
+    if (!kShards || p.spc == 1) {
       const bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&seg_full[0]), 0, abort_flag));
       tc_fence_after();
       // once seg_full completed every MMA is done, so the pipeline buffers are free
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
             if (c0 + j < p.T) stream_store(p, c0 + j, n_row, __uint_as_float(r[j]), bias_row);
         }
       }
-    } else {
+    } else if constexpr (kShards) {
       float run[kStreamRunCols];
 #pragma unroll
       for (int j = 0; j < kStreamRunCols; ++j) run[j] = 0.0f;
@@ -349,15 +354,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       cluster_wait_acquire();    // phase 1: every CTA of the cluster has started
       named_barrier(1, 128);     // all four warps have staged their rows
     }
-    if (multi && threadIdx.x == 0) {
-      // one bulk copy per owner: my rows of its range -> its receive slot [crank]
+    if (multi && threadIdx.x < p.csize) {
+      // one bulk copy per owner, issued by lane o: my rows of owner o's range ->
+      // its receive slot [crank] (each completes on the owner's byte count)
       const uint32_t bytes = static_cast<uint32_t>(p.T * R * 4);
-      for (int o = 0; o < p.csize; ++o) {
-        const uint32_t src = smem_u32(smem) + static_cast<uint32_t>(o) * bytes;
-        const uint32_t dst = dsmem_map(smem_u32(recv) + static_cast<uint32_t>(crank) * bytes,
-                                       static_cast<uint32_t>(o));
-        bulk_copy_to_peer(dst, src, bytes, dsmem_map(smem_u32(recv_bar), static_cast<uint32_t>(o)));
-      }
+      const int o = threadIdx.x;
+      const uint32_t src = smem_u32(smem) + static_cast<uint32_t>(o) * bytes;
+      const uint32_t dst = dsmem_map(smem_u32(recv) + static_cast<uint32_t>(crank) * bytes,
+                                     static_cast<uint32_t>(o));
+      bulk_copy_to_peer(dst, src, bytes, dsmem_map(smem_u32(recv_bar), static_cast<uint32_t>(o)));
     }
   }
   if (multi && warp == kStreamProducerWarp) cluster_wait_acquire();  // phase 1 (copies nothing)

@@ -79,13 +79,22 @@ const DeviceInfo* device_info() {
                "cudaDeviceGetAttribute"))
     return nullptr;
   if (smem < tpb::kTiledSmemBytes) return nullptr;
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem), "cudaFuncSetAttribute"))
-    return nullptr;
   // all of the unified L1 / shared storage as shared memory, so three ~65 KB
   // streaming CTAs fit on an SM (the driver's default carveout allows two)
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared), "cudaFuncSetAttribute"))
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<false>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<true>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared),
+               "cudaFuncSetAttribute"))
     return nullptr;
   if (!cuda_ok(cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -251,8 +260,9 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
-  if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel, tw, tx, p), "launch stream_gemm_kernel"))
-    return TP_ERR_CUDA;
+  const cudaError_t e = p.spc > 1 ? cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel<true>, tw, tx, p)
+                                  : cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel<false>, tw, tx, p);
+  if (!cuda_ok(e, "launch stream_gemm_kernel")) return TP_ERR_CUDA;
   return TP_OK;
 }
 
