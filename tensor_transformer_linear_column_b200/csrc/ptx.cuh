@@ -358,6 +358,26 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, uint32_t lo
       : "memory");
 }
 
+// Asynchronous stores from registers into a cluster peer's shared memory; the
+// bytes complete on the peer's mbarrier (`peer_bar`, a shared::cluster address
+// in the same CTA as `peer_dst`).  The source is registers, so the sender keeps
+// no buffer alive for them.
+__device__ __forceinline__ void st_async_f32(uint32_t peer_dst, float v, uint32_t peer_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(
+                   peer_dst),
+               "f"(v), "r"(peer_bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_async_f32x4(uint32_t peer_dst, float a, float b, float c,
+                                               float d, uint32_t peer_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(peer_dst),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(peer_bar)
+      : "memory");
+}
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (bulk copy / TMA) reads of them.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -375,15 +395,10 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t addr) {
+// 16-byte load from this CTA's shared memory (shared-window address).
+__device__ __forceinline__ float4 ld_shared_f32x4(uint32_t addr) {
   float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr)
                : "memory");

@@ -23,14 +23,15 @@
 // held in registers.  Column-parallel mode is the same kernel with one shard.
 //
 // Cross-CTA sum: CTA r of the cluster owns rows [r R, (r+1) R) of the tile
-// (R = 128 / csize).  Every CTA stages its fp32 partial per owner in its idle
-// pipeline buffers and sends each owner its rows with one bulk shared-memory
-// copy (cp.async.bulk, cluster scope) whose bytes complete on an mbarrier in
-// the owner; each owner waits for exactly those bytes, sums the csize partials
-// of its rows in a fixed order from its own shared memory, adds the bias,
-// applies the activation and stores bf16.  Nothing intermediate goes to global memory and there are no
-// atomics, so the result is bit-identical from run to run for a given shape
-// and t.
+// (R = 128 / csize).  Every CTA sends each owner its fp32 partial of the
+// owner's rows straight from registers with asynchronous remote stores
+// (st.async, cluster scope) whose bytes complete on an mbarrier in the owner;
+// each owner waits for exactly those bytes, sums the csize partials of its rows
+// in a fixed order from its own shared memory, adds the bias, applies the
+// activation and stores bf16.  A CTA keeps no buffer alive for its peers, so it
+// exits as soon as its own rows are stored.  Nothing intermediate goes to
+// global memory and there are no atomics, so the result is bit-identical from
+// run to run for a given shape and t.
 //
 // Weight traffic: a ring of 3-8 stages, deeper for CTAs that stream longer;
 // with static weights the first stages are requested before the kernel waits
@@ -74,22 +75,29 @@ constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when sp
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
 //   [0, stages * stage_bytes)   pipeline: per stage W tile (16 KB) then x tile (t_pad * 128 B)
-//   [.., + recv_bytes)          receive buffer [csize][T][R] fp32 (<= 128 * t_pad * 4 bytes)
-//   After the main loop the pipeline buffers hold the staging [owner][T][R] fp32 of this CTA's
-//   partial (so stages * stage_bytes >= 128 * T * 4 is required: T <= 128).
+//   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final, recv,
 //   tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
-__host__ __device__ inline int stream_recv_bytes(int t_pad, int csize) {
-  return csize > 1 ? t_pad * kStreamTileM * 4 : 0;
+//
+// Row stride RS of the receive buffer: T rounded up to 4 floats (one 16-byte
+// store carries four tokens of a row), plus 4 when that is a multiple of 32
+// floats, so eight consecutive rows read as float4 fall in distinct banks.
+__host__ __device__ inline int stream_recv_stride(int T) {
+  const int rs = (T + 3) / 4 * 4;
+  return rs % 32 == 0 ? rs + 4 : rs;
 }
 
-__host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, int t_pad, int csize) {
-  return stages * stage_bytes + stream_recv_bytes(t_pad, csize);
+__host__ __device__ inline int stream_recv_bytes(int T, int csize) {
+  return csize > 1 ? kStreamTileM * stream_recv_stride(T) * 4 : 0;
 }
 
-__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int t_pad, int csize) {
-  return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, t_pad, csize) +
+__host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, int T, int csize) {
+  return stages * stage_bytes + stream_recv_bytes(T, csize);
+}
+
+__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize) {
+  return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, T, csize) +
          (2 * stages + 6) * 8 + 16;
 }
 
@@ -100,6 +108,26 @@ __device__ __forceinline__ void stream_store(const StreamParams& p, int tok, int
   if (p.act == 1) v = gelu_tanh_f32(v);
   __nv_bfloat16 h = __float2bfloat16_rn(v);
   p.out[static_cast<size_t>(tok) * p.N + n] = *reinterpret_cast<uint16_t*>(&h);
+}
+
+// Send tokens [c0, c0 + 16) of this thread's row, values v, to the owner's
+// receive row at cluster address `dst_row`: four tokens per 16-byte store, one
+// at a time past the last full group.  Exactly T values per row are sent, the
+// byte count each owner waits for.
+__device__ __forceinline__ void stream_send16(uint32_t dst_row, uint32_t peer_bar, int c0, int T,
+                                              const float* v) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 4) {
+    const int tok = c0 + j;
+    const uint32_t dst = dst_row + static_cast<uint32_t>(tok * 4);
+    if (tok + 4 <= T) {
+      st_async_f32x4(dst, v[j], v[j + 1], v[j + 2], v[j + 3], peer_bar);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (tok + q < T) st_async_f32(dst + static_cast<uint32_t>(q * 4), v[j + q], peer_bar);
+    }
+  }
 }
 
 // k-block range [lo, hi) of cluster rank `crank`; never straddles a shard.
@@ -119,19 +147,23 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
   }
 }
 
-// kShards = false: one accumulation segment per CTA (spc == 1); registers are
-// bounded so three CTAs fit on an SM (six warps are granted registers as
-// eight), which lets the next call's CTAs start and prefetch weights while
-// this call drains.  kShards = true: several shards per CTA (spc >= 1).
+// Registers are granted to a CTA per group of four warps, so the six-warp CTA
+// is charged as eight; the bounds below are stated for 256 threads to make the
+// compiler budget for that.  kShards = false: one accumulation segment per CTA
+// (spc == 1), at most 85 registers so three CTAs fit on an SM, which lets the
+// next call's CTAs start and prefetch weights while this call drains.
+// kShards = true: several shards per CTA (spc > 1) folded in a register
+// running sum, at most 128 registers (two CTAs per SM).
+constexpr int kStreamRegThreads = 256;
 template <bool kShards>
-__global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
+__global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_x, const StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   float* recv = reinterpret_cast<float*>(smem + p.stages * p.stage_bytes);
-  const int data_bytes = stream_data_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize);
+  const int data_bytes = stream_data_bytes(p.stages, p.stage_bytes, p.T, p.csize);
   const bool multi = p.csize > 1;  // partials are summed across a cluster
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + data_bytes);
   uint64_t* full_bar = bars;
@@ -146,6 +178,7 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x;
+  float bias_own = 0.0f;  // bias of the row this thread finalises as owner
   const int crank = static_cast<int>(cluster_ctarank());  // == blockIdx.y
   const int R = kStreamTileM / p.csize;                   // rows each CTA finalises
 
@@ -181,8 +214,6 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
   const uint32_t tmem_d = *tmem_slot;
   // cluster phase 1: "this CTA has started" (waited on before any remote copy)
   if (multi) cluster_arrive_relaxed();
-  // the next kernel in the stream may start its own set-up now
-  grid_launch_dependents();
 
   const uint32_t x_bytes = static_cast<uint32_t>(p.t_pad) * kStreamTileK * 2;
   const uint32_t tx_bytes = kStreamWBytes + x_bytes;
@@ -223,6 +254,10 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
         issued |= 1u << s;
         phases = (phases & ~(1u << s)) | (ph << s);
       }
+      // every weight load of this CTA is in flight: the next kernel in the
+      // stream may start now and queue its own (earlier, its weight requests
+      // would slow this grid's last round trips)
+      grid_launch_dependents();
       if (*abort_flag) {
         // let copies already in flight land before the CTA can exit
         for (int s = 0; s < p.stages; ++s)
@@ -276,39 +311,58 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
     __syncwarp();
     if (multi) cluster_wait_acquire();  // phase 1 (this warp copies nothing)
   } else {
-    // ---------------- warps 0-3: drain TMEM, fold shards in order, stage rows per owner
+    // ---------------- warps 0-3: drain TMEM, fold shards in order, send rows to their owners
     grid_dependency_wait();
     const int row = warp * 32 + lane;  // TMEM lane == weight row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    // staging (the idle pipeline buffers): [owner][tok][row % R] fp32
-    float* stage_row = reinterpret_cast<float*>(smem) + (row / R) * p.T * R + (row % R);
     // single-CTA cluster: this thread's row is final, store it directly
     const int n_row = n_tile * kStreamTileM + row;
     const float bias_row = (!multi && p.bias != nullptr && n_row < p.N) ? bf16_to_f32(p.bias[n_row]) : 0.0f;
-    if (!kShards || p.spc == 1) {
+    // owner rows: item e of the final sum is row e % R, and R divides 128, so
+    // each thread finalises one row and can fetch its bias now, off the tail
+    const int n_own = n_tile * kStreamTileM + crank * R + static_cast<int>(threadIdx.x) % R;
+    bias_own = (multi && p.bias != nullptr && n_own < p.N) ? bf16_to_f32(p.bias[n_own]) : 0.0f;
+    uint32_t dst_row = 0u, peer_bar = 0u;
+    if (multi) {
+      // phase 1: every CTA of the cluster has started, so its receive barrier is armed
+      cluster_wait_acquire();
+      const uint32_t owner = static_cast<uint32_t>(row / R);
+      const int RS = stream_recv_stride(p.T);
+      dst_row = dsmem_map(smem_u32(recv) + static_cast<uint32_t>(((crank * R + row % R) * RS) * 4),
+                          owner);
+      peer_bar = dsmem_map(smem_u32(recv_bar), owner);
+    }
+    if constexpr (!kShards) {
       const bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&seg_full[0]), 0, abort_flag));
       tc_fence_after();
-      // once seg_full completed every MMA is done, so the pipeline buffers are free
-      for (int c0 = 0; c0 < p.T; c0 += 16) {
-        uint32_t r[16];
+      // 32 tokens per round: two TMEM loads in flight, one wait
+      for (int c0 = 0; c0 < p.T; c0 += 32) {
+        const bool two = c0 + 16 < p.T;
+        uint32_t r0[16], r1[16];
         if (ok && nkb > 0) {
-          tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0), r);
+          tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0), r0);
+          if (two) tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0 + 16), r1);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = 0u;
+          for (int j = 0; j < 16; ++j) r0[j] = r1[j] = 0u;
+        }
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          v[j] = __uint_as_float(r0[j]);
+          v[16 + j] = __uint_as_float(r1[j]);
         }
         if (multi) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < p.T) stage_row[(c0 + j) * R] = __uint_as_float(r[j]);
+          stream_send16(dst_row, peer_bar, c0, p.T, v);
+          if (two) stream_send16(dst_row, peer_bar, c0 + 16, p.T, v + 16);
         } else if (n_row < p.N) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < p.T) stream_store(p, c0 + j, n_row, __uint_as_float(r[j]), bias_row);
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < p.T) stream_store(p, c0 + j, n_row, v[j], bias_row);
         }
       }
-    } else if constexpr (kShards) {
+    } else {
       float run[kStreamRunCols];
 #pragma unroll
       for (int j = 0; j < kStreamRunCols; ++j) run[j] = 0.0f;
@@ -338,10 +392,14 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&seg_empty[region]));
       }
+      if (!ok) {
+#pragma unroll
+        for (int j = 0; j < kStreamRunCols; ++j) run[j] = 0.0f;
+      }
       if (multi) {
 #pragma unroll
-        for (int c = 0; c < kStreamRunCols; ++c)
-          if (c < p.T) stage_row[c * R] = ok ? run[c] : 0.0f;
+        for (int c = 0; c < kStreamRunCols; c += 16)
+          if (c < p.T) stream_send16(dst_row, peer_bar, c, p.T, run + c);
       } else if (n_row < p.N) {
 #pragma unroll
         for (int c = 0; c < kStreamRunCols; ++c)
@@ -349,90 +407,63 @@ __global__ void __launch_bounds__(kStreamThreads, kShards ? 1 : 3)
       }
     }
     tc_fence_before();
-    if (multi) {
-      fence_proxy_async_smem();  // staging is read by the bulk-copy engine
-      cluster_wait_acquire();    // phase 1: every CTA of the cluster has started
-      named_barrier(1, 128);     // all four warps have staged their rows
-    }
-    if (multi && threadIdx.x < p.csize) {
-      // one bulk copy per owner, issued by lane o: my rows of owner o's range ->
-      // its receive slot [crank] (each completes on the owner's byte count)
-      const uint32_t bytes = static_cast<uint32_t>(p.T * R * 4);
-      const int o = threadIdx.x;
-      const uint32_t src = smem_u32(smem) + static_cast<uint32_t>(o) * bytes;
-      const uint32_t dst = dsmem_map(smem_u32(recv) + static_cast<uint32_t>(crank) * bytes,
-                                     static_cast<uint32_t>(o));
-      bulk_copy_to_peer(dst, src, bytes, dsmem_map(smem_u32(recv_bar), static_cast<uint32_t>(o)));
-    }
   }
-  if (multi && warp == kStreamProducerWarp) cluster_wait_acquire();  // phase 1 (copies nothing)
+  if (multi && warp == kStreamProducerWarp) cluster_wait_acquire();  // phase 1 (sends nothing)
 
   __syncthreads();
   if (warp == kStreamMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_d, tcols_alloc);
   }
-  if (!multi) return;
-  if (warp >= 4) cluster_arrive_release();  // phase 2 for the warps that receive nothing
+  if (!multi || warp >= 4) return;
 
-  // ---------------- owner: fixed-order sum of the csize partials of its rows
-  if (warp < 4) {
-    // every peer always issues its copy, so this completes within microseconds
-    if (!drain_wait(smem_u32(recv_bar), 0, 50ull * 1000ull * 1000ull))
-      atomicOr(&g_tp_device_error, kErrTimeout);
-    // phase 2: my incoming copies have landed (so the peers' sources were read)
-    cluster_arrive_release();
-    const int groups4 = R / 4;
-    const int total = groups4 * p.T;
-    for (int e = threadIdx.x; e < total; e += 128) {
-      const int tok = e / groups4;
-      const int q4 = (e % groups4) * 4;
-      float4 v[8];
+  // ---------------- owner: fixed-order sum of the csize partials of its rows.
+  // Every peer always sends its T values per row, so this completes within
+  // microseconds; once it has, nothing in the cluster touches this CTA's shared
+  // memory again and the CTA may exit without a closing cluster barrier.
+  if (!drain_wait(smem_u32(recv_bar), 0, 50ull * 1000ull * 1000ull))
+    atomicOr(&g_tp_device_error, kErrTimeout);
+  const int RS = stream_recv_stride(p.T);
+  const int groups = (p.T + 3) / 4;  // four tokens of one row per item
+  const int n0 = n_tile * kStreamTileM + crank * R;
+  // csize, R = 128 / csize and jsplit = csize / shards are powers of two
+  const int r_shift = __ffs(R) - 1;
+  const uint32_t recv_s = smem_u32(recv);
+  const int j_mask = p.jsplit - 1;
+  for (int e = threadIdx.x; e < R * groups; e += 128) {
+    const int lr = e & (R - 1);
+    const int tok0 = (e >> r_shift) * 4;
+    float4 v[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c < p.csize)
-          v[c] = *reinterpret_cast<const float4*>(recv + (c * p.T + tok) * R + q4);
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f), ps = y;
+    for (int c = 0; c < 8; ++c)
+      if (c < p.csize) v[c] = ld_shared_f32x4(recv_s + static_cast<uint32_t>(((c * R + lr) * RS + tok0) * 4));
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f), ps = y;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c < p.csize) {
-          const int jj = c % p.jsplit;
-          if (jj == 0) {
-            ps = v[c];
+    for (int c = 0; c < 8; ++c) {
+      if (c < p.csize) {
+        const int jj = c & j_mask;
+        if (jj == 0) {
+          ps = v[c];
+        } else {
+          ps.x += v[c].x; ps.y += v[c].y; ps.z += v[c].z; ps.w += v[c].w;
+        }
+        if (jj == j_mask) {
+          if (c == j_mask) {
+            y = ps;
           } else {
-            ps.x += v[c].x; ps.y += v[c].y; ps.z += v[c].z; ps.w += v[c].w;
-          }
-          if (jj == p.jsplit - 1) {
-            if (c == p.jsplit - 1) {
-              y = ps;
-            } else {
-              y.x += ps.x; y.y += ps.y; y.z += ps.z; y.w += ps.w;
-            }
+            y.x += ps.x; y.y += ps.y; y.z += ps.z; y.w += ps.w;
           }
         }
-      }
-      const int n = n_tile * kStreamTileM + crank * R + q4;
-      if (n < p.N) {
-        float o[4] = {y.x, y.y, y.z, y.w};
-        if (p.bias != nullptr) {
-          const uint2 bb = *reinterpret_cast<const uint2*>(p.bias + n);
-          o[0] += __uint_as_float(bb.x << 16);
-          o[1] += __uint_as_float(bb.x & 0xFFFF0000u);
-          o[2] += __uint_as_float(bb.y << 16);
-          o[3] += __uint_as_float(bb.y & 0xFFFF0000u);
-        }
-        if (p.act == 1) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) o[q] = gelu_tanh_f32(o[q]);
-        }
-        uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-        *reinterpret_cast<uint2*>(p.out + static_cast<size_t>(tok) * p.N + n) = packed;
       }
     }
+    const int n = n0 + lr;
+    if (n < p.N) {
+      const float o[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (tok0 + q < p.T) stream_store(p, tok0 + q, n, o[q], bias_own);
+    }
   }
-  // phase 2: every CTA's incoming copies have landed, so this CTA's staging
-  // (the source of its outgoing copies) is no longer read and it may exit
-  cluster_wait_acquire();
 }
 
 }  // namespace tpb

@@ -222,7 +222,7 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
     int lo, hi;
     tpb::stream_cta_range(p, 0, lo, hi);
     const int budget =
-        (hi - lo >= 16 ? 110 : 72) * 1024 - tpb::stream_recv_bytes(p.t_pad, p.csize);
+        (hi - lo >= 16 ? 110 : 72) * 1024 - tpb::stream_recv_bytes(p.T, p.csize);
     int stages = budget / p.stage_bytes;
     stages = stages < 3 ? 3 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
     p.stages = stages;
@@ -234,12 +234,10 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
   // large T: the receive buffer leaves room for two stages only
   while (p.stages > 2 &&
-         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize) > dev.max_smem)
+         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize) > dev.max_smem)
     --p.stages;
-  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.t_pad, p.csize);
-  // the idle pipeline buffers must hold the staged partial [128][T] fp32
-  if (smem > dev.max_smem || (p.csize > 1 && p.stages * p.stage_bytes < tpb::kStreamTileM * T * 4))
-    return TP_ERR_UNSUPPORTED;
+  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize);
+  if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
 
   CUtensorMap tw, tx;
   if (!make_tmap(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), tpb::kStreamTileM))
