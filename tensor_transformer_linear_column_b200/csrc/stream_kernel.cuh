@@ -13,6 +13,12 @@
 // 128) and a contiguous range of the reduction dimension; the `csize` CTAs
 // that share an n-tile form one thread-block cluster.
 //
+// Issue rate: one thread issues a tcgen05.mma (any N up to 256) about every
+// 140 cycles, so with a handful of tokens the tensor pipe is bound by MMA
+// issue, not arithmetic: 4 KB of weight per instruction.  Two warps therefore
+// issue MMAs, one for the even and one for the odd pipeline stages, into two
+// accumulators that the epilogue adds in a fixed order.
+//
 // Row-parallel mode (the all-reduce of the row-parallel layer, done on chip):
 // the reduction dimension is cut into t shards.  Either a shard is split over
 // `jsplit` consecutive CTAs (csize = t * jsplit), or a CTA owns `spc`
@@ -38,7 +44,8 @@
 // for the preceding grid, overlapping that grid's tail.
 //
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
-// push and reduce; warp 4 issues TMA; one thread of warp 5 issues MMAs.
+// push and reduce; warp 4 issues TMA; one thread each of warps 5 and 6 issues
+// MMAs.
 #pragma once
 
 #include "ptx.cuh"
@@ -56,6 +63,7 @@ struct StreamParams {
   int shards;     // shards of the reduction dimension (1 for column-parallel)
   int t_pad;      // MMA N: tokens rounded up to 16
   int tmem_cols;  // columns of one TMEM region (power of two >= max(32, t_pad))
+  int kpb;        // k-blocks per TMA box and pipeline stage (1 or 2)
   int stages;     // smem pipeline depth (<= 8)
   int stage_bytes;
   int act;        // tp_act
@@ -64,19 +72,20 @@ struct StreamParams {
   uint16_t* out;         // [T, N]
 };
 
-constexpr int kStreamThreads = 192;
+constexpr int kStreamThreads = 224;
 constexpr int kStreamProducerWarp = 4;
-constexpr int kStreamMmaWarp = 5;
+constexpr int kStreamMmaWarp = 5;   // MMA issuers: warps 5 and 6
+constexpr int kStreamMmaWarps = 2;
 constexpr int kStreamTileM = 128;
 constexpr int kStreamTileK = 64;
-constexpr int kStreamWBytes = kStreamTileM * kStreamTileK * 2;  // 16 KB
 constexpr int kStreamMaxStages = 8;
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
-//   [0, stages * stage_bytes)   pipeline: per stage W tile (16 KB) then x tile (t_pad * 128 B)
+//   [0, stages * stage_bytes)   pipeline: per stage kpb W tiles (16 KB each) then kpb x
+//                               tiles (t_pad * 128 B each)
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
-//   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final, recv,
+//   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
 //   tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
 //
@@ -98,7 +107,7 @@ __host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, in
 
 __host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize) {
   return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, T, csize) +
-         (2 * stages + 6) * 8 + 16;
+         (2 * stages + 7) * 8 + 16;
 }
 
 // Epilogue of one value: bias, activation, round to bf16, store.
@@ -147,9 +156,9 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
   }
 }
 
-// Registers are granted to a CTA per group of four warps, so the six-warp CTA
-// is charged as eight; the bounds below are stated for 256 threads to make the
-// compiler budget for that.  kShards = false: one accumulation segment per CTA
+// Registers are granted to a CTA per group of four warps, so the seven-warp
+// CTA is charged as eight; the bounds below are stated for 256 threads to make
+// the compiler budget for that.  kShards = false: one accumulation segment per CTA
 // (spc == 1), at most 85 registers so three CTAs fit on an SM, which lets the
 // next call's CTAs start and prefetch weights while this call drains.
 // kShards = true: several shards per CTA (spc > 1) folded in a register
@@ -170,8 +179,8 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   uint64_t* empty_bar = bars + p.stages;
   uint64_t* seg_full = bars + 2 * p.stages;       // [2]
   uint64_t* seg_empty = bars + 2 * p.stages + 2;  // [2]
-  uint64_t* final_bar = bars + 2 * p.stages + 4;
-  uint64_t* recv_bar = bars + 2 * p.stages + 5;  // bytes of the peers' partials for my rows
+  uint64_t* final_bar = bars + 2 * p.stages + 4;  // [2], one per MMA issuer
+  uint64_t* recv_bar = bars + 2 * p.stages + 6;   // bytes of the peers' partials for my rows
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -185,8 +194,12 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   int kb_lo, kb_hi;
   stream_cta_range(p, crank, kb_lo, kb_hi);
   const int nkb = kb_hi - kb_lo;
-  const int kb_seg = nkb / p.spc;  // k-blocks per accumulation segment
-  const uint32_t tcols_alloc = static_cast<uint32_t>(p.spc > 1 ? 2 * p.tmem_cols : p.tmem_cols);
+  const int kpb = p.kpb;            // k-blocks per box (divides every CTA's range)
+  const int nbox = nkb / kpb;       // boxes (pipeline stages' worth) of this CTA
+  const int box_seg = nbox / p.spc;  // boxes per accumulation segment
+  // two TMEM regions: the two issuers' accumulators (one segment), or
+  // alternate shards (several segments)
+  const uint32_t tcols_alloc = static_cast<uint32_t>(2 * p.tmem_cols);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -194,10 +207,11 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&seg_full[b]), 1);
+      // one segment: both issuers commit to seg_full[0]
+      mbar_init(smem_u32(&seg_full[b]), kShards ? 1 : kStreamMmaWarps);
       mbar_init(smem_u32(&seg_empty[b]), 4);
+      mbar_init(smem_u32(&final_bar[b]), 1);
     }
-    mbar_init(smem_u32(final_bar), 1);
     mbar_init(smem_u32(recv_bar), 1);
     // expect csize partials of T x R fp32 before any peer can send (phase 1)
     mbar_arrive_expect_tx(smem_u32(recv_bar), static_cast<uint32_t>(p.csize * p.T * R * 4));
@@ -216,7 +230,9 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   if (multi) cluster_arrive_relaxed();
 
   const uint32_t x_bytes = static_cast<uint32_t>(p.t_pad) * kStreamTileK * 2;
-  const uint32_t tx_bytes = kStreamWBytes + x_bytes;
+  const uint32_t w_bytes = kStreamTileM * kStreamTileK * 2;  // one k-block of W: 16 KB
+  const uint32_t xoff = static_cast<uint32_t>(kpb) * w_bytes;  // x tiles follow the W tiles
+  const uint32_t tx_bytes = static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
 
   if (warp == kStreamProducerWarp) {
     if (lane == 0) {
@@ -228,31 +244,36 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       uint32_t issued = 0u, phases = 0u;  // per stage: a load was issued / its phase bit
       // weights are read-only model parameters: with prefetch_w the first
       // stages' weight tiles are requested before the preceding grid finishes
-      const int pre = p.prefetch_w ? (nkb < p.stages ? nkb : p.stages) : 0;
+      // box i holds k-blocks kb_lo + i kpb .. + kpb - 1 (3-D maps: column in
+      // the block, row, k-block)
+      const int pre = p.prefetch_w ? (nbox < p.stages ? nbox : p.stages) : 0;
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[i]), tx_bytes);
-        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[i]), (kb_lo + i) * kStreamTileK, w_row,
-                         pol_w);
+        tma_load_3d_hint(st, &tmap_w, smem_u32(&full_bar[i]), 0, w_row, kb_lo + i * kpb, pol_w);
         issued |= 1u << i;
       }
       grid_dependency_wait();  // activations may come from the preceding grid
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
-        tma_load_2d(st + kStreamWBytes, &tmap_x, smem_u32(&full_bar[i]),
-                    (kb_lo + i) * kStreamTileK, 0);
+        tma_load_3d(st + xoff, &tmap_x, smem_u32(&full_bar[i]), 0, 0, kb_lo + i * kpb);
       }
-      for (int i = pre; i < nkb; ++i) {
-        const int s = i % p.stages;
-        const uint32_t ph = static_cast<uint32_t>(i / p.stages) & 1u;
+      // stage s and pass parity ph of box i, advanced without divisions
+      int s = pre == p.stages ? 0 : pre;
+      uint32_t ph = pre == p.stages ? 1u : 0u;
+      for (int i = pre; i < nbox; ++i) {
         if (!wait_parity(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag)) break;
         const uint32_t st = smem_u32(smem + s * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[s]), tx_bytes);
-        const int kc = (kb_lo + i) * kStreamTileK;
-        tma_load_2d_hint(st, &tmap_w, smem_u32(&full_bar[s]), kc, w_row, pol_w);
-        tma_load_2d(st + kStreamWBytes, &tmap_x, smem_u32(&full_bar[s]), kc, 0);
+        const int kb = kb_lo + i * kpb;
+        tma_load_3d_hint(st, &tmap_w, smem_u32(&full_bar[s]), 0, w_row, kb, pol_w);
+        tma_load_3d(st + xoff, &tmap_x, smem_u32(&full_bar[s]), 0, 0, kb);
         issued |= 1u << s;
         phases = (phases & ~(1u << s)) | (ph << s);
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       // every weight load of this CTA is in flight: the next kernel in the
       // stream may start now and queue its own (earlier, its weight requests
@@ -266,15 +287,23 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       }
     }
     __syncwarp();
-  } else if (warp == kStreamMmaWarp) {
-    if (lane == 0) {
-      // ---------------- MMA issuer: spc segments, segment g into TMEM region g % 2
+  } else if (warp >= kStreamMmaWarp) {
+    const int me = warp - kStreamMmaWarp;  // issuer 0 or 1
+    if (lane == 0 && (!kShards || me == 0)) {
+      // ---------------- MMA issuers.  One segment: issuer j takes the boxes in
+      // the odd (j = 1) or even (j = 0) pipeline stages, into TMEM region j;
+      // each stage has a single consumer, so its fills are taken in order.
+      // Several segments (one issuer): segment g into region g % 2.
       const uint32_t idesc = idesc_bf16_f32(kStreamTileM, p.t_pad);
+      // descriptors of stage 0; a byte offset b within the ring adds b >> 4
+      const uint64_t desc0 = desc_kmajor_sw128(smem_u32(smem));
       bool ok = true;
-      int i = 0;
+      int i = 0;        // box index
+      int s = 0;        // its stage
+      uint32_t ph = 0u;  // its pass parity
       for (int g = 0; ok && g < p.spc; ++g) {
-        const int region = g & 1;
-        if (g >= 2) {
+        const int region = kShards ? (g & 1) : me;
+        if (kShards && g >= 2) {
           if (!wait_parity(smem_u32(&seg_empty[region]), static_cast<uint32_t>((g >> 1) - 1) & 1u,
                            abort_flag)) {
             ok = false;
@@ -283,33 +312,44 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
           tc_fence_after();
         }
         const uint32_t d = tmem_d + static_cast<uint32_t>(region * p.tmem_cols);
-        for (int kb = 0; kb < kb_seg; ++kb, ++i) {
-          const int s = i % p.stages;
-          const uint32_t ph = static_cast<uint32_t>(i / p.stages) & 1u;
-          if (!wait_parity(smem_u32(&full_bar[s]), ph, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + s * p.stage_bytes);
+        const int end = (g + 1) * box_seg;
+        bool first = true;
+        for (; i < end; ++i) {
+          if (kShards || (s & 1) == me) {
+            if (!wait_parity(smem_u32(&full_bar[s]), ph, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t st = static_cast<uint32_t>(s * p.stage_bytes);
+            for (int c = 0; c < kpb; ++c) {
+              const uint64_t da = desc0 + ((st + static_cast<uint32_t>(c) * w_bytes) >> 4);
+              const uint64_t db = desc0 + ((st + xoff + static_cast<uint32_t>(c) * x_bytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
-            umma_bf16(d, desc_kmajor_sw128(st + kk * 32),
-                      desc_kmajor_sw128(st + kStreamWBytes + kk * 32), idesc,
-                      (kb > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
+                umma_bf16(d, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2),
+                          idesc, first ? 0u : 1u);
+                first = false;
+              }
+            }
+            umma_commit(smem_u32(&empty_bar[s]));
           }
-          umma_commit(smem_u32(&empty_bar[s]));
+          if (++s == p.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
-        if (ok) umma_commit(smem_u32(&seg_full[region]));
+        // an issuer without boxes commits at once; its region is not read
+        if (ok) umma_commit(smem_u32(&seg_full[kShards ? region : 0]));
       }
       if (!ok) {
         // every MMA issued so far must finish before TMEM / smem are released
-        umma_commit(smem_u32(final_bar));
-        drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
+        umma_commit(smem_u32(&final_bar[me]));
+        drain_wait(smem_u32(&final_bar[me]), 0, 50ull * 1000ull * 1000ull);
       }
     }
     __syncwarp();
-    if (multi) cluster_wait_acquire();  // phase 1 (this warp copies nothing)
+    if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
     // ---------------- warps 0-3: drain TMEM, fold shards in order, send rows to their owners
     grid_dependency_wait();
@@ -335,23 +375,30 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     if constexpr (!kShards) {
       const bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&seg_full[0]), 0, abort_flag));
       tc_fence_after();
+      // the issuers' accumulators that received a box, added in issuer order
+      const int na = ok ? (nbox < kStreamMmaWarps ? nbox : kStreamMmaWarps) : 0;
       // 32 tokens per round: two TMEM loads in flight, one wait
       for (int c0 = 0; c0 < p.T; c0 += 32) {
         const bool two = c0 + 16 < p.T;
-        uint32_t r0[16], r1[16];
-        if (ok && nkb > 0) {
-          tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0), r0);
-          if (two) tmem_ld16(tmem_d + lane_addr + static_cast<uint32_t>(c0 + 16), r1);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) r0[j] = r1[j] = 0u;
-        }
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = __uint_as_float(r0[j]);
-          v[16 + j] = __uint_as_float(r1[j]);
+        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+        for (int a = 0; a < na; ++a) {
+          uint32_t r0[16], r1[16];
+          const uint32_t col = tmem_d + lane_addr + static_cast<uint32_t>(a * p.tmem_cols + c0);
+          tmem_ld16(col, r0);
+          if (two) {
+            tmem_ld16(col + 16u, r1);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r1[j] = 0u;
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v[j] = a == 0 ? __uint_as_float(r0[j]) : v[j] + __uint_as_float(r0[j]);
+            v[16 + j] = a == 0 ? __uint_as_float(r1[j]) : v[16 + j] + __uint_as_float(r1[j]);
+          }
         }
         if (multi) {
           stream_send16(dst_row, peer_bar, c0, p.T, v);

@@ -138,6 +138,25 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
   return ok;
 }
 
+// 3-D view of a row-major [rows, cols] bf16 matrix as (column within a
+// 64-column block, row, block): a box {64, box_rows, blocks} lands in shared
+// memory as `blocks` consecutive 128-byte-swizzled [box_rows][64] tiles.
+bool make_tmap_blocks(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows, uint32_t blocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_ok(cudaErrorSymbolNotFound, "cuTensorMapEncodeTiled lookup");
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (blocks)");
+  return ok;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool feat_ok(int n) { return n > 0 && n % 64 == 0; }
 inline int next_pow2(int v) {
@@ -170,12 +189,13 @@ struct StreamGeometry {
   int csize = 0, jsplit = 0, spc = 0;
 };
 
-// Cluster shape of the streaming kernel for n_tiles output tiles: the largest
-// cluster (1, 2, 4 or 8 CTAs along K) that keeps the grid within two CTAs per
-// SM, so every CTA is resident from the start.  Either a shard is split over
-// jsplit CTAs or a CTA owns spc whole shards (register running sum: t_pad <= 64).
-// csize == 0 when no shape fits.
-StreamGeometry stream_geometry(int n_tiles, int kb_total, int shards, int t_pad, int sms) {
+// Cluster shape of the streaming kernel for an N x K weight in 128-row tiles:
+// the largest cluster (1, 2, 4 or 8 CTAs along K) that keeps the grid within
+// two CTAs per SM, so every CTA is resident from the start.  Either a shard is
+// split over jsplit CTAs or a CTA owns spc whole shards (register running sum:
+// t_pad <= 64).  csize == 0 when no shape fits.
+StreamGeometry stream_geometry(int N, int kb_total, int shards, int t_pad, int sms) {
+  const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
   StreamGeometry fallback;
   const int kbs = kb_total / shards;
   for (int csize = 8; csize >= 1; csize >>= 1) {
@@ -210,22 +230,37 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   p.kb_total = K / tpb::kStreamTileK;
   p.t_pad = (T + 15) / 16 * 16;
   p.tmem_cols = next_pow2(p.t_pad < 32 ? 32 : p.t_pad);
-  p.stage_bytes = tpb::kStreamWBytes + p.t_pad * tpb::kStreamTileK * 2;
+  p.stage_bytes = (tpb::kStreamTileM + p.t_pad) * tpb::kStreamTileK * 2;
   p.shards = shards;
   p.csize = geo.csize;
   p.jsplit = geo.jsplit;
   p.spc = geo.spc;
-  // Ring depth: CTAs that stream >= 16 k-blocks get ~110 KB (two CTAs per SM,
-  // deep ring); short streams get ~72 KB so three CTAs fit on an SM and the
-  // next kernel's CTAs can start while this one drains.  At least 3 stages.
+  // Ring depth: CTAs that stream >= 256 KB of weights get ~110 KB (two CTAs
+  // per SM, deep ring); short streams get ~72 KB so three CTAs fit on an SM
+  // and the next kernel's CTAs can start while this one drains.  At least 3
+  // k-blocks in flight.  Two k-blocks per TMA box where every CTA's range is
+  // even and three such stages fit the budget: a CTA's boxes complete one
+  // after another, so larger boxes stream faster, but only a ring that still
+  // holds three of them keeps enough in flight.
   {
     int lo, hi;
     tpb::stream_cta_range(p, 0, lo, hi);
-    const int budget =
-        (hi - lo >= 16 ? 110 : 72) * 1024 - tpb::stream_recv_bytes(p.T, p.csize);
-    int stages = budget / p.stage_bytes;
-    stages = stages < 3 ? 3 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
+    const long w_cta = static_cast<long>(hi - lo) * tpb::kStreamTileM * tpb::kStreamTileK * 2;
+    const int budget = (w_cta >= 256 * 1024 ? 110 : 72) * 1024 -
+                       tpb::stream_recv_bytes(p.T, p.csize);
+    const int kb_bytes = p.stage_bytes;  // one k-block of W and x
+    bool even = p.spc == 1;
+    for (int r = 0; even && r < p.csize; ++r) {
+      tpb::stream_cta_range(p, r, lo, hi);
+      even = lo % 2 == 0 && hi % 2 == 0;
+    }
+    p.kpb = (even && 6 * kb_bytes <= budget) ? 2 : 1;
+    int kbs = budget / kb_bytes;
+    kbs = kbs < 3 ? 3 : kbs;
+    int stages = kbs / p.kpb;
+    stages = stages < 2 ? 2 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
     p.stages = stages;
+    p.stage_bytes = p.kpb * kb_bytes;
   }
   p.act = act;
   p.prefetch_w = prefetch_weights();
@@ -240,10 +275,11 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
 
   CUtensorMap tw, tx;
-  if (!make_tmap(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), tpb::kStreamTileM))
+  if (!make_tmap_blocks(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                        static_cast<uint32_t>(tpb::kStreamTileM), static_cast<uint32_t>(p.kpb)))
     return TP_ERR_CUDA;
-  if (!make_tmap(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(K),
-                 static_cast<uint32_t>(p.t_pad)))
+  if (!make_tmap_blocks(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(K),
+                        static_cast<uint32_t>(p.t_pad), static_cast<uint32_t>(p.kpb)))
     return TP_ERR_CUDA;
 
   cudaLaunchConfig_t cfg{};
@@ -369,7 +405,7 @@ tp_status run_colpar(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T
   if (dev == nullptr) return TP_ERR_CUDA;
   if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
-    const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, 1, t_pad, dev->sms);
+    const StreamGeometry g = stream_geometry(N, K / 64, 1, t_pad, dev->sms);
     if (g.csize > 0) return launch_stream(*dev, g, x, w, b, T, K, N, 1, act, out, stream);
   }
   return launch_tiled(*dev, x, w, b, T, K, N, 1, act, out, stream);
@@ -381,7 +417,7 @@ tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T
   if (dev == nullptr) return TP_ERR_CUDA;
   if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
-    const StreamGeometry g = stream_geometry((N + 127) / 128, K / 64, t, t_pad, dev->sms);
+    const StreamGeometry g = stream_geometry(N, K / 64, t, t_pad, dev->sms);
     if (g.csize > 0) return launch_stream(*dev, g, h, w, b, T, K, N, t, 0, out, stream);
   }
   return launch_tiled(*dev, h, w, b, T, K, N, t, 0, out, stream);
