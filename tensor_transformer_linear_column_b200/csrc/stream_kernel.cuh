@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       const uint32_t idesc = idesc_bf16_f32(kStreamTileM, p.t_pad);
       // descriptors of stage 0; a byte offset b within the ring adds b >> 4
       const uint64_t desc0 = desc_kmajor_sw128(smem_u32(smem));
+      // every stage needs activations from the preceding grid: park in the
+      // hardware wait instead of polling the first stage while it drains
+      grid_dependency_wait();
       bool ok = true;
       int i = 0;        // box index
       int s = 0;        // its stage

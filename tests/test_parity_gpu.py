@@ -128,7 +128,9 @@ def test_sq4096_colpar(sq_weights, T, path):
 RAGGED_COL = [(1, 64, 64), (2, 768, 64), (3, 576, 320), (3, 256, 1088), (5, 4096, 320),
               (8, 512, 64), (17, 128, 1088), (63, 192, 256), (65, 64, 320),
               (128, 256, 384), (130, 320, 576), (200, 256, 1024), (257, 128, 320),
-              (300, 64, 1088), (5, 256, 20480), (40, 128, 20480)]
+              (300, 64, 1088), (5, 256, 20480), (40, 128, 20480),
+              # long per-CTA streams: two k-blocks per TMA box, an odd number of stages
+              (3, 8192, 320), (9, 16384, 192)]
 
 
 @pytest.mark.parametrize("T,K,N", RAGGED_COL)
@@ -150,7 +152,7 @@ def test_colpar_ragged(T, K, N, act):
 RAGGED_ROW = [(1, 512, 64, 1), (5, 512, 320, 2), (33, 1024, 256, 4), (64, 512, 128, 8),
               (128, 1024, 192, 4), (129, 2048, 320, 8), (300, 512, 64, 4), (7, 576, 192, 3),
               (40, 1024, 256, 16), (2, 4096, 128, 2), (3, 768, 320, 3), (6, 4096, 64, 16),
-              (8, 2048, 1088, 8), (1, 256, 64, 1)]
+              (8, 2048, 1088, 8), (1, 256, 64, 1), (2, 8192, 192, 2)]
 
 
 @pytest.mark.parametrize("T,K,N,t", RAGGED_ROW)
