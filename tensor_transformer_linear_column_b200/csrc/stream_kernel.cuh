@@ -64,6 +64,7 @@ struct StreamParams {
   int t_pad;      // MMA N: tokens rounded up to 16
   int tmem_cols;  // columns of one TMEM region (power of two >= max(32, t_pad))
   int kpb;        // k-blocks per TMA box and pipeline stage (1 or 2)
+  int l2_ahead;   // boxes after the ring's first fill prefetched into L2 before the grid wait
   int stages;     // smem pipeline depth (<= 8)
   int stage_bytes;
   int act;        // tp_act
@@ -252,6 +253,13 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         mbar_arrive_expect_tx(smem_u32(&full_bar[i]), tx_bytes);
         tma_load_3d_hint(st, &tmap_w, smem_u32(&full_bar[i]), 0, w_row, kb_lo + i * kpb, pol_w);
         issued |= 1u << i;
+      }
+      // the next l2_ahead boxes go to L2 only: a short look-ahead keeps HBM
+      // busy while the preceding grid drains; a longer one delays this grid's
+      // own first loads
+      if (p.prefetch_w) {
+        const int l2_end = nbox < pre + p.l2_ahead ? nbox : pre + p.l2_ahead;
+        for (int i = pre; i < l2_end; ++i) tma_prefetch_l2_3d(&tmap_w, 0, w_row, kb_lo + i * kpb);
       }
       grid_dependency_wait();  // activations may come from the preceding grid
       for (int i = 0; i < pre; ++i) {
