@@ -80,6 +80,7 @@ constexpr int kStreamMmaWarps = 2;
 constexpr int kStreamTileM = 128;
 constexpr int kStreamTileK = 64;
 constexpr int kStreamMaxStages = 8;
+constexpr int kStreamReleaseBack = 2;  // boxes still to issue when the next grid is released
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
@@ -261,6 +262,13 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         const int l2_end = nbox < pre + p.l2_ahead ? nbox : pre + p.l2_ahead;
         for (int i = pre; i < l2_end; ++i) tma_prefetch_l2_3d(&tmap_w, 0, w_row, kb_lo + i * kpb);
       }
+      // the next kernel in the stream is released once this CTA has issued
+      // all but its last kStreamReleaseBack weight boxes: earlier, its weight
+      // requests slow this grid's last round trips; later, its own weight
+      // prefetch starts too late to cover this grid's tail
+      const int release_at = nbox - 1 - kStreamReleaseBack;
+      bool released = release_at < pre;
+      if (released) grid_launch_dependents();
       grid_dependency_wait();  // activations may come from the preceding grid
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
@@ -282,11 +290,12 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
           s = 0;
           ph ^= 1u;
         }
+        if (i == release_at) {
+          grid_launch_dependents();
+          released = true;
+        }
       }
-      // every weight load of this CTA is in flight: the next kernel in the
-      // stream may start now and queue its own (earlier, its weight requests
-      // would slow this grid's last round trips)
-      grid_launch_dependents();
+      if (!released) grid_launch_dependents();  // the loop stopped early
       if (*abort_flag) {
         // let copies already in flight land before the CTA can exit
         for (int s = 0; s < p.stages; ++s)
