@@ -63,20 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Same, letting the hardware suspend the thread for up to `ns` nanoseconds
-// while the phase is incomplete (it resumes as soon as the phase completes).
-__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(bar), "r"(parity), "r"(ns)
-      : "memory");
-  return done != 0;
-}
-
 // Wait until the phase of `bar` with parity `parity` has completed.
 // Returns false (after flagging the error and raising *abort) if the wait runs
 // past the limit, or at once if *abort is already raised by another role.
@@ -123,16 +109,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Same, with an L2 eviction-priority hint (weights are streamed once).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int c0, int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
-      : "memory");
-}
-
 // 3-D tile load: coordinates (c0 innermost, c1, c2), completion on `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2) {
@@ -163,12 +139,6 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
@@ -379,24 +349,8 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Bulk copy of `bytes` (multiple of 16, 16-byte aligned ends) from this CTA's
-// shared memory to a cluster peer's shared memory; completion is counted in
-// bytes on the mbarrier `peer_bar` in the destination CTA.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, uint32_t local_src,
-                                                  uint32_t bytes, uint32_t peer_bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(peer_dst),
-      "r"(local_src), "r"(bytes), "r"(peer_bar)
-      : "memory");
 }
 
 // Asynchronous stores from registers into a cluster peer's shared memory; the
@@ -417,16 +371,6 @@ __device__ __forceinline__ void st_async_f32x4(uint32_t peer_dst, float a, float
           "r"(peer_dst),
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(peer_bar)
       : "memory");
-}
-
-// Order this thread's generic-proxy shared-memory writes before later
-// async-proxy (bulk copy / TMA) reads of them.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // Address of the same shared-memory offset in cluster CTA `rank`.

@@ -39,9 +39,11 @@
 // global memory and there are no atomics, so the result is bit-identical from
 // run to run for a given shape and t.
 //
-// Weight traffic: a ring of 3-8 stages, deeper for CTAs that stream longer;
-// with static weights the first stages are requested before the kernel waits
-// for the preceding grid, overlapping that grid's tail.
+// Weight traffic: a ring of 2-8 stages of one or two k-blocks each (3-D TMA
+// boxes), deeper for CTAs that stream longer.  With static weights the first
+// ring's worth is requested before the kernel waits for the preceding grid,
+// and CTAs with short streams send the next two boxes to L2, overlapping that
+// grid's tail.
 //
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
 // push and reduce; warp 4 issues TMA; one thread each of warps 5 and 6 issues
