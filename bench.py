@@ -2,12 +2,13 @@
 """Benchmark of the tensor-parallel block on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload sq4096|tiny|mlp70b|attn70b|mlp405b] [--tp T]
+                    [--workload sq4096|tiny|mlp70b|mlp70b_w8|attn70b|mlp405b] [--tp T]
 
 Default workload: the pages' TP=2 square projection (W[4096, 4096] split by
 columns into 2 shards), decode batches T = 1, 8 and 64.  One step = one pass of
 the block's path over one batch of each T (3 column-parallel calls, 73 tokens).
-The other workloads are available for measurement with --workload.
+The other workloads are available for measurement with --workload
+(mlp70b_w8: the 70B-shaped MLP with 8-bit E4M3 weights and per-row scales).
 
 Timing: W warm-up steps, then exactly K steps captured in CUDA graphs and
 bracketed by a barrier + synchronize on both sides, timed with CUDA events on
@@ -217,6 +218,19 @@ class Workload:
                          None if d["b2"] is None else d["b2"].to(device))
             self.ws = torch.empty(max(tp.tp_mlp_workspace_bytes(T, cfg.ffn) for T in self.Ts),
                                   dtype=torch.uint8, device=device)
+        elif name == "mlp70b_w8":
+            self.t = tp_degree or cfg.tp_degrees[-1]
+            self.Ts = list(cfg.tokens)
+            d = workloads.mlp_inputs(cfg, self.Ts[0])
+            self.xs = {T: workloads.mlp_x(cfg, T) for T in self.Ts}
+            q1, s1 = workloads.quantize_e4m3_rows(d["w1"])
+            q2, s2 = workloads.quantize_e4m3_rows(d["w2"])
+            self.weight_bytes = q1.numel() + q2.numel() + 4 * (s1.numel() + s2.numel())
+            self.hidden_in = self.hidden_out = cfg.hidden
+            self.weights = [tuple(a.to(device) for a in (q1, s1, q2, s2))]
+            self.bias = (None, None)
+            self.ws = torch.empty(max(tp.tp_mlp_workspace_bytes(T, cfg.ffn) for T in self.Ts),
+                                  dtype=torch.uint8, device=device)
         elif name == "attn70b":
             self.t = tp_degree or cfg.tp_degrees[0]
             self.Ts = list(cfg.tokens)
@@ -256,6 +270,9 @@ class Workload:
             w = self.weights[(i * len(self.Ts) + j) % self.rot]
             if self.name == "sq4096":
                 tp.tp_colpar_gemm_gelu(xs[T], w, None, self.t, "none", out=outs[T])
+            elif self.name == "mlp70b_w8":
+                tp.tp_mlp_forward_w8(xs[T], w[0], w[1], None, w[2], w[3], None, self.t,
+                                     self.cfg.act, out=outs[T], workspace=self.ws)
             elif self.name == "attn70b":
                 tp.tp_attn_proj_forward(xs[T], w[0], None, self.ctx, w[1], None,
                                         self.cfg.n_q_heads, self.cfg.n_kv_heads,
@@ -270,11 +287,12 @@ class Workload:
         b = 0
         for T in self.Ts:
             b += self.weight_bytes + 2 * T * (self.hidden_in + self.hidden_out)
-            if self.name in ("tiny", "mlp70b", "mlp405b"):
+            if self.name in ("tiny", "mlp70b", "mlp70b_w8", "mlp405b"):
                 b += 2 * 2 * T * self.cfg.ffn  # h written and read once
         return b
 
     def step_flops(self):
+        """2 T per weight element (bf16 weights: 2 bytes per element)."""
         f = 0
         for T in self.Ts:
             f += 2 * T * self.weight_bytes // 2
@@ -317,6 +335,10 @@ class _OracleRunner:
             T0 = cfg.tokens[0]
             d = workloads.mlp_inputs(cfg, T0)
             self.w1, self.w2, self.b1, self.b2 = d["w1"], d["w2"], d["b1"], d["b2"]
+            if cfg.weights == "e4m3":
+                import oracle
+                self.w1 = oracle.E4M3Weight(*workloads.quantize_e4m3_rows(d["w1"]))
+                self.w2 = oracle.E4M3Weight(*workloads.quantize_e4m3_rows(d["w2"]))
             if cfg.sample_rows:
                 rows = workloads.sample_rows(T0, cfg.sample_rows)
                 self.xs = {T0: d["x"][rows]}
@@ -428,6 +450,8 @@ def workload_config(name, t, wl):
         "sq4096": "column-parallel projection W[4096,4096] bf16, t=2 column shards, decode T=1,8,64",
         "tiny": "MLP block H=256 F=1024, t=2, GeLU, biases, T=8",
         "mlp70b": "Llama-3-70B-shaped MLP decode H=8192 F=28672, GeLU, T=1,16,64",
+        "mlp70b_w8": "Llama-3-70B-shaped MLP decode H=8192 F=28672, GeLU, T=1,16,64, "
+                     "8-bit weights (FP8 E4M3 codes, one fp32 scale per row)",
         "attn70b": "Llama-3-70B-shaped attention projections prefill T=4096, QKV 8192->10240 "
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
         "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192",

@@ -206,6 +206,41 @@ tp_status tp_mlp_forward_noalloc(const tp_bf16* x, const tp_bf16* w1, const tp_b
                                  int T, int H, int F, int tp_degree, int act,
                                  tp_bf16* out, tp_stream_t stream);
 
+/*
+ * 8-bit weights (decode).  In decode every token reads every weight, so the
+ * weight bytes set the time per token; the pages' example reads a 70B model
+ * in 8-bit (drpranayjha.com "AI Infrastructure series, Part 5", section
+ * "Reason 2: one user's answers are too slow").  These calls take each weight
+ * as FP8 E4M3 bytes (the OCP "E4M3FN" encoding: sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits, no infinities, S.1111.111 = NaN) with one fp32
+ * scale per output row:
+ *   W[n, k] = w_scale[n] * e4m3(w8[n, k])
+ * and otherwise compute exactly what the bf16 calls compute with that W:
+ * bf16 activations, fp32 accumulation (every E4M3 value is a bf16 value, so
+ * the products are the bf16 kernel's), the scale applied to the fp32 sum of
+ * each output before bias and activation.
+ *   w8       [N, K] (w1: [F, H], w2: [H, F]) bytes, row-major, 16-byte aligned
+ *   w_scale  [N] fp32 (s1: [F], s2: [H]), 16-byte aligned
+ * Other arguments, checks and errors as tp_colpar_gemm_gelu,
+ * tp_rowpar_gemm_reduce and tp_mlp_forward.  These calls always use the
+ * weight-streaming kernel: T <= 128 (else TP_ERR_UNSUPPORTED); row-parallel
+ * calls whose shards would not fit two per streaming CTA also return
+ * TP_ERR_UNSUPPORTED (none of t <= 8 at the 70B shapes).
+ */
+tp_status tp_colpar_gemm_gelu_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,
+                                 const tp_bf16* b, int T, int K, int N, int tp_degree, int act,
+                                 tp_bf16* out, tp_stream_t stream);
+
+tp_status tp_rowpar_gemm_reduce_w8(const tp_bf16* h, const uint8_t* w8, const float* w_scale,
+                                   const tp_bf16* b, int T, int K, int N, int tp_degree,
+                                   tp_bf16* out, tp_stream_t stream);
+
+tp_status tp_mlp_forward_w8(const tp_bf16* x, const uint8_t* w1, const float* s1,
+                            const tp_bf16* b1, const uint8_t* w2, const float* s2,
+                            const tp_bf16* b2, int T, int H, int F, int tp_degree, int act,
+                            tp_bf16* out, void* workspace, size_t workspace_bytes,
+                            tp_stream_t stream);
+
 /* A short English description of a status code (static storage). */
 const char* tp_status_string(tp_status status);
 

@@ -4,10 +4,13 @@ Importable only from the tests, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline / reference leg.  The CUDA product path never touches it.
 """
 from .tp_oracle import (  # noqa: F401
+    E4M3_TABLE,
+    E4M3Weight,
     apply_act,
     attn_out,
     attn_qkv,
     colpar_linear,
+    e4m3_value,
     gelu_tanh,
     heads_divisible,
     linear,

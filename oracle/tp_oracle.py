@@ -38,11 +38,19 @@ Memory: large weights are upcast to float64 a block of *output features* at a
 time.  That only bounds memory; every output element is still one dot product
 over its full reduction dimension.
 
+8-bit weights (drpranayjha.com "AI Infrastructure series, Part 5", "Reason 2":
+decode reads 8-bit weights): an ``E4M3Weight`` holds FP8 E4M3 codes and one
+scale per output row, W[n, k] = scale[n] * e4m3(q[n, k]); every function here
+that takes a weight also takes one, and reads it through its exact float64
+values (the E4M3 code table is written out from the format's definition in
+``e4m3_value``).
+
 Pinned by tests/test_oracle.py against: brute-force math.fsum dot products on
 tiny inputs, torch's own tanh-GeLU in float64 and the erf GeLU (a different
 formula that the tanh form approximates), the odd-part identity of GeLU, the
-shard-sum and shard-concatenation invariants for every t, and special cases
-(identity weights, one-hot inputs, t = 1).
+shard-sum and shard-concatenation invariants for every t, special cases
+(identity weights, one-hot inputs, t = 1), and, for 8-bit weights, the E4M3
+format's landmark values and torch's own float8_e4m3fn decoding.
 """
 from __future__ import annotations
 
@@ -65,8 +73,51 @@ GELU_CUBIC = 0.044715
 _OUT_BLOCK = 2048
 
 
+def e4m3_value(code: int) -> float:
+    """The value of one FP8 E4M3 code ("E4M3FN"): 1 sign bit, 4 exponent bits
+    with bias 7, 3 mantissa bits; exponent field 0 is subnormal (m/8 * 2^-6);
+    there are no infinities and S.1111.111 is NaN."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+class E4M3Weight:
+    """An 8-bit weight [N, K]: codes q (uint8) and row scales (float32),
+    W[n, k] = scale[n] * e4m3(q[n, k]).  Slicing by rows, or by rows and
+    columns, gives the matching sub-weight; ``to_f64`` decodes it exactly."""
+
+    def __init__(self, q: ArrayLike, scale: ArrayLike):
+        self.q = q
+        self.scale = scale
+        self.shape = tuple(int(d) for d in q.shape)
+
+    def __getitem__(self, idx):
+        rows = idx[0] if isinstance(idx, tuple) else idx
+        return E4M3Weight(self.q[idx], self.scale[rows])
+
+    def dequant(self) -> np.ndarray:
+        if torch is not None and isinstance(self.q, torch.Tensor):
+            codes = self.q.detach().to("cpu").numpy()
+        else:
+            codes = np.asarray(self.q)
+        sc = to_f64(self.scale)
+        return E4M3_TABLE[codes.astype(np.int64)] * sc[:, None]
+
+
 def to_f64(a: ArrayLike) -> np.ndarray:
-    """Exact upcast of a bf16/fp32/fp64 tensor or array to a float64 ndarray."""
+    """Exact upcast of a bf16/fp32/fp64 tensor or array (or an 8-bit weight)
+    to a float64 ndarray."""
+    if isinstance(a, E4M3Weight):
+        return a.dequant()
     if torch is not None and isinstance(a, torch.Tensor):
         return a.detach().to("cpu").to(torch.float64).numpy()
     return np.asarray(a, dtype=np.float64)

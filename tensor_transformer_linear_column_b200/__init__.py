@@ -45,6 +45,9 @@ SIGNATURES = {
     "tp_mlp_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "tp_colpar_gemm_gelu_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "tp_rowpar_gemm_reduce_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "tp_mlp_forward_w8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_status_string": (ctypes.c_char_p, [_I]),
     "tp_last_cuda_error": (ctypes.c_char_p, []),
     "tp_device_error_check": (_I, []),
@@ -99,6 +102,22 @@ def _ptr(t: Optional[torch.Tensor], name: str, dev: torch.device) -> Optional[in
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != torch.bfloat16:
         raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _ptr_typed(t: Optional[torch.Tensor], name: str, dev: torch.device,
+               dtype: torch.dtype) -> Optional[int]:
+    """Like _ptr for the 8-bit weight bytes (uint8) and their fp32 scales."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.device != dev:
         raise ValueError(f"{name} is on {t.device}, expected {dev}")
     if not t.is_contiguous():
@@ -184,6 +203,80 @@ def tp_mlp_forward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor]
                                int(tp_degree), _act(act), _ptr(out, "out", dev),
                                workspace.data_ptr(), ws_bytes, _stream(stream))
     _check(st, "tp_mlp_forward")
+    return out
+
+
+def tp_colpar_gemm_gelu_w8(x: torch.Tensor, w8: torch.Tensor, w_scale: torch.Tensor,
+                           b: Optional[torch.Tensor], tp_degree: int, act="none",
+                           out: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """tp_colpar_gemm_gelu with an 8-bit weight: w8 [N, K] E4M3 bytes (uint8) and
+    w_scale [N] fp32, W[n, k] = w_scale[n] * e4m3(w8[n, k])."""
+    T, K = x.shape
+    N = w8.shape[0]
+    if w8.shape[1] != K or tuple(w_scale.shape) != (N,):
+        raise ValueError("w8 must be [N, K] and w_scale [N]")
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    st = load().tp_colpar_gemm_gelu_w8(
+        _ptr(x, "x", dev), _ptr_typed(w8, "w8", dev, torch.uint8),
+        _ptr_typed(w_scale, "w_scale", dev, torch.float32), _ptr(b, "b", dev), T, K, N,
+        int(tp_degree), _act(act), _ptr(out, "out", dev), _stream(stream))
+    _check(st, "tp_colpar_gemm_gelu_w8")
+    return out
+
+
+def tp_rowpar_gemm_reduce_w8(h: torch.Tensor, w8: torch.Tensor, w_scale: torch.Tensor,
+                             b: Optional[torch.Tensor], tp_degree: int,
+                             out: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """tp_rowpar_gemm_reduce with an 8-bit weight (see tp_colpar_gemm_gelu_w8)."""
+    T, K = h.shape
+    N = w8.shape[0]
+    if w8.shape[1] != K or tuple(w_scale.shape) != (N,):
+        raise ValueError("w8 must be [N, K] and w_scale [N]")
+    dev = h.device
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    st = load().tp_rowpar_gemm_reduce_w8(
+        _ptr(h, "h", dev), _ptr_typed(w8, "w8", dev, torch.uint8),
+        _ptr_typed(w_scale, "w_scale", dev, torch.float32), _ptr(b, "b", dev), T, K, N,
+        int(tp_degree), _ptr(out, "out", dev), _stream(stream))
+    _check(st, "tp_rowpar_gemm_reduce_w8")
+    return out
+
+
+def tp_mlp_forward_w8(x: torch.Tensor, w1: torch.Tensor, s1: torch.Tensor,
+                      b1: Optional[torch.Tensor], w2: torch.Tensor, s2: torch.Tensor,
+                      b2: Optional[torch.Tensor], tp_degree: int, act="gelu_tanh",
+                      out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """tp_mlp_forward with 8-bit weights: w1 [F, H] and w2 [H, F] E4M3 bytes,
+    s1 [F] and s2 [H] fp32 row scales."""
+    T, H = x.shape
+    F = w1.shape[0]
+    if w1.shape[1] != H or tuple(w2.shape) != (H, F):
+        raise ValueError("w1 must be [F, H] and w2 [H, F]")
+    if tuple(s1.shape) != (F,) or tuple(s2.shape) != (H,):
+        raise ValueError("s1 must be [F] and s2 [H]")
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    need = tp_mlp_workspace_bytes(T, F)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the same device")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load().tp_mlp_forward_w8(
+        _ptr(x, "x", dev), _ptr_typed(w1, "w1", dev, torch.uint8),
+        _ptr_typed(s1, "s1", dev, torch.float32), _ptr(b1, "b1", dev),
+        _ptr_typed(w2, "w2", dev, torch.uint8), _ptr_typed(s2, "s2", dev, torch.float32),
+        _ptr(b2, "b2", dev), T, H, F, int(tp_degree), _act(act), _ptr(out, "out", dev),
+        workspace.data_ptr(), ws_bytes, _stream(stream))
+    _check(st, "tp_mlp_forward_w8")
     return out
 
 

@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 namespace tpb {
@@ -422,6 +424,28 @@ __device__ __forceinline__ float gelu_tanh_f32(float z) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Eight FP8 E4M3 values (byte k of q = element k) to eight bf16 values
+// (element k in bits [16 (k % 2), +16) of word k / 2).  E4M3 -> f16 is exact,
+// and every E4M3 value is also exact in bf16.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 q) {
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t word = j < 2 ? q.x : q.y;
+    const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(word >> (16 * (j & 1)));
+    const __half2 h(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3));
+    const float2 f = __half22float2(h);
+    w[j] = pack_bf16x2(f.x, f.y);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (tcgen05.mma operands, bulk copies).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

@@ -45,9 +45,18 @@
 // and CTAs with short streams send the next two boxes to L2, overlapping that
 // grid's tail.
 //
+// 8-bit weights (kW8): the weight is FP8 E4M3 with one fp32 scale per row
+// (drpranayjha.com "AI Infrastructure series, Part 5", section "Reason 2":
+// decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 into a
+// staging buffer; the four epilogue warps, idle while the weights stream,
+// rewrite it as the bf16 tile the MMA reads (exact: every E4M3 value is a bf16
+// value), and the row scale multiplies the fp32 sum before bias and activation.
+// The MMAs and everything after them are those of the bf16 kernel; HBM traffic
+// is halved.
+//
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
-// push and reduce; warp 4 issues TMA; one thread each of warps 5 and 6 issues
-// MMAs.
+// push and reduce, and with 8-bit weights first convert the weight tiles;
+// warp 4 issues TMA; one thread each of warps 5 and 6 issues MMAs.
 #pragma once
 
 #include "ptx.cuh"
@@ -72,6 +81,7 @@ struct StreamParams {
   int act;        // tp_act
   int prefetch_w; // weights may be read before the preceding grid completes
   const uint16_t* bias;  // [N] or nullptr
+  const float* w_scale;  // [N] row scales of an 8-bit weight (kW8), else unused
   uint16_t* out;         // [T, N]
 };
 
@@ -81,16 +91,18 @@ constexpr int kStreamMmaWarp = 5;   // MMA issuers: warps 5 and 6
 constexpr int kStreamMmaWarps = 2;
 constexpr int kStreamTileM = 128;
 constexpr int kStreamTileK = 64;
+constexpr int kStreamW8Bytes = kStreamTileM * kStreamTileK;  // one k-block of 8-bit W: 8 KB
 constexpr int kStreamMaxStages = 8;
 constexpr int kStreamReleaseBack = 2;  // boxes still to issue when the next grid is released
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
 //   [0, stages * stage_bytes)   pipeline: per stage kpb W tiles (16 KB each) then kpb x
-//                               tiles (t_pad * 128 B each)
+//                               tiles (t_pad * 128 B each); with 8-bit weights (kpb = 1)
+//                               then the 8 KB E4M3 staging tile [128][64] bytes
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
-//   tmem slot, abort flag
+//   conv[stages] (8-bit weights: tile converted), tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
 //
 // Row stride RS of the receive buffer: T rounded up to 4 floats (one 16-byte
@@ -111,7 +123,7 @@ __host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, in
 
 __host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize) {
   return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, T, csize) +
-         (2 * stages + 7) * 8 + 16;
+         (3 * stages + 7) * 8 + 16;
 }
 
 // Epilogue of one value: bias, activation, round to bf16, store.
@@ -168,7 +180,7 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
 // kShards = true: several shards per CTA (spc > 1) folded in a register
 // running sum, at most 128 registers (two CTAs per SM).
 constexpr int kStreamRegThreads = 256;
-template <bool kShards>
+template <bool kShards, bool kW8>
 __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_x, const StreamParams p) {
@@ -185,13 +197,15 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   uint64_t* seg_empty = bars + 2 * p.stages + 2;  // [2]
   uint64_t* final_bar = bars + 2 * p.stages + 4;  // [2], one per MMA issuer
   uint64_t* recv_bar = bars + 2 * p.stages + 6;   // bytes of the peers' partials for my rows
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
+  uint64_t* conv_bar = bars + 2 * p.stages + 7;   // [stages]: 8-bit tile converted to bf16
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv_bar + p.stages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x;
-  float bias_own = 0.0f;  // bias of the row this thread finalises as owner
+  float bias_own = 0.0f;   // bias of the row this thread finalises as owner
+  float scale_own = 1.0f;  // and its 8-bit weight scale
   const int crank = static_cast<int>(cluster_ctarank());  // == blockIdx.y
   const int R = kStreamTileM / p.csize;                   // rows each CTA finalises
 
@@ -209,6 +223,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
+      mbar_init(smem_u32(&conv_bar[s]), 4);  // one arrive per converting warp
     }
     for (int b = 0; b < 2; ++b) {
       // one segment: both issuers commit to seg_full[0]
@@ -236,7 +251,11 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   const uint32_t x_bytes = static_cast<uint32_t>(p.t_pad) * kStreamTileK * 2;
   const uint32_t w_bytes = kStreamTileM * kStreamTileK * 2;  // one k-block of W: 16 KB
   const uint32_t xoff = static_cast<uint32_t>(kpb) * w_bytes;  // x tiles follow the W tiles
-  const uint32_t tx_bytes = static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
+  // 8-bit weights (kpb == 1): the E4M3 tile lands in staging after x
+  const uint32_t w8off = w_bytes + x_bytes;
+  const uint32_t wdst = kW8 ? w8off : 0u;
+  const uint32_t tx_bytes =
+      kW8 ? kStreamW8Bytes + x_bytes : static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
 
   if (warp == kStreamProducerWarp) {
     if (lane == 0) {
@@ -254,7 +273,8 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = smem_u32(smem + i * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[i]), tx_bytes);
-        tma_load_3d_hint(st, &tmap_w, smem_u32(&full_bar[i]), 0, w_row, kb_lo + i * kpb, pol_w);
+        tma_load_3d_hint(st + wdst, &tmap_w, smem_u32(&full_bar[i]), 0, w_row, kb_lo + i * kpb,
+                         pol_w);
         issued |= 1u << i;
       }
       // the next l2_ahead boxes go to L2 only: a short look-ahead keeps HBM
@@ -284,7 +304,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         const uint32_t st = smem_u32(smem + s * p.stage_bytes);
         mbar_arrive_expect_tx(smem_u32(&full_bar[s]), tx_bytes);
         const int kb = kb_lo + i * kpb;
-        tma_load_3d_hint(st, &tmap_w, smem_u32(&full_bar[s]), 0, w_row, kb, pol_w);
+        tma_load_3d_hint(st + wdst, &tmap_w, smem_u32(&full_bar[s]), 0, w_row, kb, pol_w);
         tma_load_3d(st + xoff, &tmap_x, smem_u32(&full_bar[s]), 0, 0, kb);
         issued |= 1u << s;
         phases = (phases & ~(1u << s)) | (ph << s);
@@ -338,7 +358,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         bool first = true;
         for (; i < end; ++i) {
           if (kShards || (s & 1) == me) {
-            if (!wait_parity(smem_u32(&full_bar[s]), ph, abort_flag)) {
+            if (!wait_parity(smem_u32(kW8 ? &conv_bar[s] : &full_bar[s]), ph, abort_flag)) {
               ok = false;
               break;
             }
@@ -373,6 +393,35 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     __syncwarp();
     if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
+    if constexpr (kW8) {
+      // ---------------- warps 0-3, first: E4M3 -> bf16.  Thread t rewrites row
+      // t of every box's weight tile, 8 elements (16 bytes) at a time, into the
+      // 128-byte-swizzled layout of a TMA tile (16-byte chunk j of row t at
+      // chunk j ^ (t % 8)), which the MMA descriptor expects.
+      const int t = static_cast<int>(threadIdx.x);
+      int s = 0;
+      uint32_t ph = 0u;
+      bool ok = true;
+      for (int i = 0; i < nbox; ++i) {
+        ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
+        if (ok) {
+          const uint8_t* src = smem + s * p.stage_bytes + w8off + t * kStreamTileK;
+          uint8_t* dst = smem + s * p.stage_bytes + t * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint2 q = *reinterpret_cast<const uint2*>(src + j * 8);
+            *reinterpret_cast<uint4*>(dst + ((j ^ (t & 7)) * 16)) = e4m3x8_to_bf16x8(q);
+          }
+          fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&conv_bar[s]));
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
     // ---------------- warps 0-3: drain TMEM, fold shards in order, send rows to their owners
     grid_dependency_wait();
     const int row = warp * 32 + lane;  // TMEM lane == weight row within the tile
@@ -380,10 +429,12 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     // single-CTA cluster: this thread's row is final, store it directly
     const int n_row = n_tile * kStreamTileM + row;
     const float bias_row = (!multi && p.bias != nullptr && n_row < p.N) ? bf16_to_f32(p.bias[n_row]) : 0.0f;
+    const float scale_row = (kW8 && !multi && n_row < p.N) ? p.w_scale[n_row] : 1.0f;
     // owner rows: item e of the final sum is row e % R, and R divides 128, so
     // each thread finalises one row and can fetch its bias now, off the tail
     const int n_own = n_tile * kStreamTileM + crank * R + static_cast<int>(threadIdx.x) % R;
     bias_own = (multi && p.bias != nullptr && n_own < p.N) ? bf16_to_f32(p.bias[n_own]) : 0.0f;
+    scale_own = (kW8 && multi && n_own < p.N) ? p.w_scale[n_own] : 1.0f;
     uint32_t dst_row = 0u, peer_bar = 0u;
     if (multi) {
       // phase 1: every CTA of the cluster has started, so its receive barrier is armed
@@ -428,7 +479,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         } else if (n_row < p.N) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (c0 + j < p.T) stream_store(p, c0 + j, n_row, v[j], bias_row);
+            if (c0 + j < p.T) stream_store(p, c0 + j, n_row, kW8 ? v[j] * scale_row : v[j], bias_row);
         }
       }
     } else {
@@ -472,7 +523,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       } else if (n_row < p.N) {
 #pragma unroll
         for (int c = 0; c < kStreamRunCols; ++c)
-          if (c < p.T) stream_store(p, c, n_row, run[c], bias_row);
+          if (c < p.T) stream_store(p, c, n_row, kW8 ? run[c] * scale_row : run[c], bias_row);
       }
     }
     tc_fence_before();
@@ -530,7 +581,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       const float o[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (tok0 + q < p.T) stream_store(p, tok0 + q, n, o[q], bias_own);
+        if (tok0 + q < p.T) stream_store(p, tok0 + q, n, kW8 ? o[q] * scale_own : o[q], bias_own);
     }
   }
 }

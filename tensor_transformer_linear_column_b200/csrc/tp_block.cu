@@ -66,6 +66,18 @@ EncodeTiledFn encode_fn() {
 }
 
 // Per-device facts and one-time kernel attributes.  Returns nullptr on failure.
+using StreamKernel = void (*)(const CUtensorMap, const CUtensorMap, const tpb::StreamParams);
+
+// Largest dynamic shared memory, and all of the unified L1 / shared storage
+// as shared memory, for one instantiation of the streaming kernel.
+bool stream_attrs(StreamKernel k, int smem) {
+  return cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                 "cudaFuncSetAttribute") &&
+         cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      cudaSharedmemCarveoutMaxShared),
+                 "cudaFuncSetAttribute");
+}
+
 const DeviceInfo* device_info() {
   int dev = 0;
   if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -81,20 +93,10 @@ const DeviceInfo* device_info() {
   if (smem < tpb::kTiledSmemBytes) return nullptr;
   // all of the unified L1 / shared storage as shared memory, so three ~65 KB
   // streaming CTAs fit on an SM (the driver's default carveout allows two)
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-               "cudaFuncSetAttribute") ||
-      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-               "cudaFuncSetAttribute") ||
-      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<false>,
-                                    cudaFuncAttributePreferredSharedMemoryCarveout,
-                                    cudaSharedmemCarveoutMaxShared),
-               "cudaFuncSetAttribute") ||
-      !cuda_ok(cudaFuncSetAttribute(tpb::stream_gemm_kernel<true>,
-                                    cudaFuncAttributePreferredSharedMemoryCarveout,
-                                    cudaSharedmemCarveoutMaxShared),
-               "cudaFuncSetAttribute"))
+  if (!stream_attrs(tpb::stream_gemm_kernel<false, false>, smem) ||
+      !stream_attrs(tpb::stream_gemm_kernel<true, false>, smem) ||
+      !stream_attrs(tpb::stream_gemm_kernel<false, true>, smem) ||
+      !stream_attrs(tpb::stream_gemm_kernel<true, true>, smem))
     return nullptr;
   if (!cuda_ok(cudaFuncSetAttribute(tpb::tiled_gemm_kernel<false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -154,6 +156,24 @@ bool make_tmap_blocks(CUtensorMap* map, const void* base, uint64_t rows, uint64_
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (blocks)");
+  return ok;
+}
+
+// Same view of a row-major [rows, cols] 8-bit matrix, unswizzled: a box
+// {64, box_rows, 1} lands as [box_rows][64] bytes.
+bool make_tmap_blocks_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_ok(cudaErrorSymbolNotFound, "cuTensorMapEncodeTiled lookup");
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols, 64};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (8-bit blocks)");
   return ok;
 }
 
@@ -219,10 +239,14 @@ StreamGeometry stream_geometry(int N, int kb_total, int shards, int t_pad, int s
 
 // Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
 // sum (1 for the column-parallel layer).  Requires T <= 128 and a geometry
-// from stream_geometry().
+// from stream_geometry().  With `w_scale` non-null the weight is 8-bit (E4M3
+// bytes, [N, K]) and w_scale[n] scales row n; the geometry must then keep
+// spc <= 2 (both shard regions are drained after all tiles are converted).
 tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const tp_bf16* x,
-                        const tp_bf16* w, const tp_bf16* b, int T, int K, int N, int shards,
-                        int act, tp_bf16* out, cudaStream_t stream) {
+                        const void* w, const float* w_scale, const tp_bf16* b, int T, int K,
+                        int N, int shards, int act, tp_bf16* out, cudaStream_t stream) {
+  const bool w8 = w_scale != nullptr;
+  if (w8 && geo.spc > 2) return TP_ERR_UNSUPPORTED;
   StreamParams p{};
   p.T = T;
   p.K = K;
@@ -245,16 +269,18 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   {
     int lo, hi;
     tpb::stream_cta_range(p, 0, lo, hi);
-    const long w_cta = static_cast<long>(hi - lo) * tpb::kStreamTileM * tpb::kStreamTileK * 2;
+    const long w_cta =
+        static_cast<long>(hi - lo) * tpb::kStreamTileM * tpb::kStreamTileK * (w8 ? 1 : 2);
     const int budget = (w_cta >= 256 * 1024 ? 110 : 72) * 1024 -
                        tpb::stream_recv_bytes(p.T, p.csize);
-    const int kb_bytes = p.stage_bytes;  // one k-block of W and x
+    // one k-block of W (bf16) and x, plus its 8 KB staging tile for 8-bit W
+    const int kb_bytes = p.stage_bytes + (w8 ? tpb::kStreamW8Bytes : 0);
     bool even = p.spc == 1;
     for (int r = 0; even && r < p.csize; ++r) {
       tpb::stream_cta_range(p, r, lo, hi);
       even = lo % 2 == 0 && hi % 2 == 0;
     }
-    p.kpb = (even && 6 * kb_bytes <= budget) ? 2 : 1;
+    p.kpb = (!w8 && even && 6 * kb_bytes <= budget) ? 2 : 1;
     int kbs = budget / kb_bytes;
     kbs = kbs < 3 ? 3 : kbs;
     int stages = kbs / p.kpb;
@@ -269,6 +295,7 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   p.act = act;
   p.prefetch_w = prefetch_weights();
   p.bias = b;
+  p.w_scale = w_scale;
   p.out = out;
   const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
   // large T: the receive buffer leaves room for two stages only
@@ -279,9 +306,12 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
 
   CUtensorMap tw, tx;
-  if (!make_tmap_blocks(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
-                        static_cast<uint32_t>(tpb::kStreamTileM), static_cast<uint32_t>(p.kpb)))
-    return TP_ERR_CUDA;
+  const bool tw_ok =
+      w8 ? make_tmap_blocks_u8(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                               static_cast<uint32_t>(tpb::kStreamTileM))
+         : make_tmap_blocks(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                            static_cast<uint32_t>(tpb::kStreamTileM), static_cast<uint32_t>(p.kpb));
+  if (!tw_ok) return TP_ERR_CUDA;
   if (!make_tmap_blocks(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(K),
                         static_cast<uint32_t>(p.t_pad), static_cast<uint32_t>(p.kpb)))
     return TP_ERR_CUDA;
@@ -298,8 +328,11 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
-  const cudaError_t e = p.spc > 1 ? cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel<true>, tw, tx, p)
-                                  : cudaLaunchKernelEx(&cfg, tpb::stream_gemm_kernel<false>, tw, tx, p);
+  StreamKernel k = p.spc > 1 ? (w8 ? tpb::stream_gemm_kernel<true, true>
+                                   : tpb::stream_gemm_kernel<true, false>)
+                             : (w8 ? tpb::stream_gemm_kernel<false, true>
+                                   : tpb::stream_gemm_kernel<false, false>);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tw, tx, p);
   if (!cuda_ok(e, "launch stream_gemm_kernel")) return TP_ERR_CUDA;
   return TP_OK;
 }
@@ -410,7 +443,7 @@ tp_status run_colpar(const tp_bf16* x, const tp_bf16* w, const tp_bf16* b, int T
   if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
     const StreamGeometry g = stream_geometry(N, K / 64, 1, t_pad, dev->sms);
-    if (g.csize > 0) return launch_stream(*dev, g, x, w, b, T, K, N, 1, act, out, stream);
+    if (g.csize > 0) return launch_stream(*dev, g, x, w, nullptr, b, T, K, N, 1, act, out, stream);
   }
   return launch_tiled(*dev, x, w, b, T, K, N, 1, act, out, stream);
 }
@@ -422,9 +455,22 @@ tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T
   if (use_stream(*dev, T, N)) {
     const int t_pad = (T + 15) / 16 * 16;
     const StreamGeometry g = stream_geometry(N, K / 64, t, t_pad, dev->sms);
-    if (g.csize > 0) return launch_stream(*dev, g, h, w, b, T, K, N, t, 0, out, stream);
+    if (g.csize > 0) return launch_stream(*dev, g, h, w, nullptr, b, T, K, N, t, 0, out, stream);
   }
   return launch_tiled(*dev, h, w, b, T, K, N, t, 0, out, stream);
+}
+
+// 8-bit weights: the streaming kernel only (T <= kStreamMaxTokens).
+tp_status run_linear_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,
+                        const tp_bf16* b, int T, int K, int N, int shards, int act, tp_bf16* out,
+                        cudaStream_t stream) {
+  if (T > kStreamMaxTokens) return TP_ERR_UNSUPPORTED;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  const int t_pad = (T + 15) / 16 * 16;
+  const StreamGeometry g = stream_geometry(N, K / 64, shards, t_pad, dev->sms);
+  if (g.csize == 0) return TP_ERR_UNSUPPORTED;
+  return launch_stream(*dev, g, x, w8, w_scale, b, T, K, N, shards, act, out, stream);
 }
 
 // ------------------------------------------------------------------ checks
@@ -509,6 +555,55 @@ tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_
   tp_status s = run_colpar(x, w_qkv, b_qkv, T, H, static_cast<int>(nqkv), TP_ACT_NONE, qkv_out, st);
   if (s != TP_OK) return s;
   return run_rowpar(ctx, w_o, b_o, T, static_cast<int>(nctx), H, tp_degree, out, st);
+}
+
+tp_status tp_colpar_gemm_gelu_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,
+                                 const tp_bf16* b, int T, int K, int N, int tp_degree, int act,
+                                 tp_bf16* out, tp_stream_t stream) {
+  tp_status s = check_linear(x, w8, b, out, T, K, N, act);
+  if (s != TP_OK) return s;
+  if (w_scale == nullptr) return TP_ERR_NULL;
+  if (!aligned16(w_scale)) return TP_ERR_ALIGN;
+  if (tp_degree < 1 || N % tp_degree != 0) return TP_ERR_TP_DEGREE;
+  return run_linear_w8(x, w8, w_scale, b, T, K, N, 1, act, out,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_rowpar_gemm_reduce_w8(const tp_bf16* h, const uint8_t* w8, const float* w_scale,
+                                   const tp_bf16* b, int T, int K, int N, int tp_degree,
+                                   tp_bf16* out, tp_stream_t stream) {
+  tp_status s = check_linear(h, w8, b, out, T, K, N, TP_ACT_NONE);
+  if (s != TP_OK) return s;
+  if (w_scale == nullptr) return TP_ERR_NULL;
+  if (!aligned16(w_scale)) return TP_ERR_ALIGN;
+  if (tp_degree < 1 || K % tp_degree != 0 || (K / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  return run_linear_w8(h, w8, w_scale, b, T, K, N, tp_degree, TP_ACT_NONE, out,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_mlp_forward_w8(const tp_bf16* x, const uint8_t* w1, const float* s1,
+                            const tp_bf16* b1, const uint8_t* w2, const float* s2,
+                            const tp_bf16* b2, int T, int H, int F, int tp_degree, int act,
+                            tp_bf16* out, void* workspace, size_t workspace_bytes,
+                            tp_stream_t stream) {
+  if (x == nullptr || w1 == nullptr || s1 == nullptr || w2 == nullptr || s2 == nullptr ||
+      out == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(s1) || !aligned16(w2) || !aligned16(s2) ||
+      !aligned16(out) || (b1 != nullptr && !aligned16(b1)) || (b2 != nullptr && !aligned16(b2)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || !feat_ok(F)) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_TANH) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || F % tp_degree != 0 || (F / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  if (T > kStreamMaxTokens) return TP_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < tp_mlp_workspace_bytes(T, F))
+    return TP_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TP_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tp_bf16* h = static_cast<tp_bf16*>(workspace);
+  tp_status s = run_linear_w8(x, w1, s1, b1, T, H, F, 1, act, h, st);
+  if (s != TP_OK) return s;
+  return run_linear_w8(h, w2, s2, b2, T, F, H, tp_degree, TP_ACT_NONE, out, st);
 }
 
 const char* tp_status_string(tp_status status) {

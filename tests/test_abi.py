@@ -114,6 +114,35 @@ def test_rowpar_rejects_bad_arguments(lib):
     assert _rowpar(lib, t=-1) == tp.TP_ERR_TP_DEGREE
 
 
+def test_w8_calls_reject_bad_arguments(lib):
+    # every check here runs before any CUDA call, so no device is needed
+    def col(x=GOOD, w=GOOD, sc=GOOD, T=8, K=256, N=1024, t=2, act=0):
+        return lib.tp_colpar_gemm_gelu_w8(x, w, sc, None, T, K, N, t, act, GOOD, None)
+
+    def row(h=GOOD, w=GOOD, sc=GOOD, T=8, K=1024, N=256, t=2):
+        return lib.tp_rowpar_gemm_reduce_w8(h, w, sc, None, T, K, N, t, GOOD, None)
+
+    def mlp(sc1=GOOD, sc2=GOOD, T=8, t=2, ws=GOOD, ws_bytes=1 << 20):
+        return lib.tp_mlp_forward_w8(GOOD, GOOD, sc1, None, GOOD, sc2, None, T, 256, 1024, t, 1,
+                                     GOOD, ws, ws_bytes, None)
+    assert col(sc=None) == tp.TP_ERR_NULL
+    assert col(w=None) == tp.TP_ERR_NULL
+    assert col(sc=ODD) == tp.TP_ERR_ALIGN
+    assert col(w=ODD) == tp.TP_ERR_ALIGN
+    assert col(K=100) == tp.TP_ERR_SHAPE
+    assert col(t=3) == tp.TP_ERR_TP_DEGREE
+    assert col(act=9) == tp.TP_ERR_UNSUPPORTED
+    assert col(T=129) == tp.TP_ERR_UNSUPPORTED        # decode path only
+    assert row(sc=None) == tp.TP_ERR_NULL
+    assert row(t=32) == tp.TP_ERR_TP_DEGREE
+    assert row(T=200) == tp.TP_ERR_UNSUPPORTED
+    assert mlp(sc2=None) == tp.TP_ERR_NULL
+    assert mlp(sc1=ODD) == tp.TP_ERR_ALIGN
+    assert mlp(t=3) == tp.TP_ERR_TP_DEGREE
+    assert mlp(T=129) == tp.TP_ERR_UNSUPPORTED
+    assert mlp(ws=None) == tp.TP_ERR_WORKSPACE
+
+
 def test_mlp_rejects_bad_arguments(lib):
     def call(ws=GOOD, ws_bytes=1 << 20, t=2, F=1024, act=1, x=GOOD):
         return lib.tp_mlp_forward(x, GOOD, None, GOOD, None, 8, 256, F, t, act, GOOD, ws,

@@ -325,3 +325,89 @@ def test_planted_dropped_partial_is_caught(monkeypatch):
             y = y + p
         return y if b is None else y + oracle.to_f64(b)[None, :]
     assert _pins_fail(monkeypatch, "shard_sum", bad) >= 1
+
+
+# ---------------------------------------------------------------- 8-bit weights
+
+def _e4m3_codes(shape, seed):
+    """Random finite E4M3 codes of both signs (NaN codes 0x7F / 0xFF excluded)."""
+    g = torch.Generator().manual_seed(seed)
+    mag = torch.randint(0, 0x7F, shape, generator=g, dtype=torch.int32)
+    sign = torch.randint(0, 2, shape, generator=g, dtype=torch.int32) * 0x80
+    return (mag | sign).to(torch.uint8)
+
+
+def test_e4m3_landmark_values():
+    # the E4M3 format's own landmarks: 1.0, the largest finite value 448, the
+    # smallest normal 2^-6, the smallest subnormal 2^-9, and the NaN codes
+    t = oracle.E4M3_TABLE
+    assert t[0x38] == 1.0 and t[0xB8] == -1.0
+    assert t[0x7E] == 448.0 and t[0xFE] == -448.0
+    assert t[0x08] == 2.0 ** -6 and t[0x01] == 2.0 ** -9 and t[0x07] == 7 * 2.0 ** -9
+    assert t[0x00] == 0.0 and math.copysign(1.0, t[0x80]) == -1.0
+    assert math.isnan(t[0x7F]) and math.isnan(t[0xFF])
+    pos = t[:0x7F]
+    assert np.all(np.diff(pos) > 0)                 # codes 0..0x7E increase strictly
+    assert np.array_equal(t[0x80:0xFF], -pos)       # the sign bit only negates
+
+
+def test_e4m3_table_matches_torch_float8():
+    # an independent decoder: torch's float8_e4m3fn
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    ref = ref.to(torch.float64).numpy()
+    t = oracle.E4M3_TABLE
+    assert np.array_equal(np.isnan(ref), np.isnan(t))
+    assert np.array_equal(ref[~np.isnan(ref)], t[~np.isnan(t)])
+
+
+def test_w8_linear_matches_fsum_bruteforce():
+    q = _e4m3_codes((6, 40), 11)
+    sc = torch.rand(6, generator=torch.Generator().manual_seed(12)) * 0.01 + 1e-3
+    x = _bf16_np((3, 40), 1.0, 13)
+    b = _bf16_np((6,), 0.1, 14)
+    w = np.array([[sc[n].item() * oracle.e4m3_value(int(q[n, k])) for k in range(40)]
+                  for n in range(6)])
+    got = oracle.linear(x, oracle.E4M3Weight(q, sc), b)
+    assert _close(got, _fsum_linear(x, w, b), np.abs(got).max() + 1.0)
+
+
+def test_w8_shards_equal_the_dequantised_weight():
+    # column and row shards of an 8-bit weight slice codes and scales together
+    q = _e4m3_codes((48, 64), 21)
+    sc = torch.rand(48, generator=torch.Generator().manual_seed(22)) * 0.01
+    wd = q.view(torch.float8_e4m3fn).to(torch.float64) * sc.to(torch.float64)[:, None]
+    x = _bf16_np((5, 64), 1.0, 23)
+    w8 = oracle.E4M3Weight(q, sc)
+    for t in (1, 2, 4):
+        a = oracle.colpar_linear(x, w8, None, t, "gelu_tanh")
+        b = oracle.colpar_linear(x, wd.numpy(), None, t, "gelu_tanh")
+        assert _close(a, b, np.abs(b).max() + 1.0)
+        h = _bf16_np((5, 48), 1.0, 24 + t)
+        wr = oracle.E4M3Weight(q.T.contiguous(), torch.ones(64))
+        a = oracle.rowpar_linear(h, wr, None, t)
+        b = oracle.rowpar_linear(h, q.T.contiguous().view(torch.float8_e4m3fn)
+                                 .to(torch.float64).numpy(), None, t)
+        assert _close(a, b, np.abs(b).max() + 1.0)
+
+
+def test_planted_wrong_e4m3_bias_is_caught(monkeypatch):
+    def bad_value(code):
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        sign = -1.0 if code & 0x80 else 1.0
+        if e == 0xF and m == 0x7:
+            return math.nan
+        if e == 0:
+            return sign * (m / 8.0) * 2.0 ** -7
+        return sign * (1.0 + m / 8.0) * 2.0 ** (e - 8)     # exponent bias 8, not 7
+    bad = np.array([bad_value(c) for c in range(256)])
+    monkeypatch.setattr(tp_oracle, "E4M3_TABLE", bad)
+    monkeypatch.setattr(oracle, "E4M3_TABLE", bad)
+    caught = 0
+    for c in (test_e4m3_landmark_values, test_e4m3_table_matches_torch_float8,
+              test_w8_shards_equal_the_dequantised_weight):
+        try:
+            c()
+        except AssertionError:
+            caught += 1
+    assert caught >= 2

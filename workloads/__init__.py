@@ -20,6 +20,13 @@ Recipe (one place, so every consumer sees the same bits):
 
 Shapes and standard deviations are the five workloads the block is measured
 on; see ``CONFIGS``.
+
+8-bit weights (``quantize_e4m3_rows``): a drawn bf16 weight is stored as FP8
+E4M3 codes with one fp32 scale per output row, scale[n] = max_k |w[n, k]| / 448
+(448 is the largest finite E4M3 value) and q[n, k] = E4M3(w[n, k] / scale[n]),
+rounded to nearest by ``Tensor.to(torch.float8_e4m3fn)``.  The layer then uses
+the weight scale[n] * e4m3(q[n, k]); the oracle and the GPU both receive q and
+the scales.
 """
 from __future__ import annotations
 
@@ -96,6 +103,7 @@ class MLPConfig:
     b_std: Optional[float]  # None -> the workload has no biases
     x_fp32: bool = False   # x drawn in fp32 and rounded by the caller
     sample_rows: Optional[int] = None  # oracle checks this many seeded rows
+    weights: str = "bf16"  # "bf16", or "e4m3": 8-bit weights with row scales
 
 
 @dataclasses.dataclass(frozen=True)
@@ -134,6 +142,10 @@ CONFIGS: Dict[str, object] = {
     # Llama-3-70B-shaped MLP decode
     "mlp70b": MLPConfig("mlp70b", hidden=8192, ffn=28672, tokens=(1, 16, 64),
                         tp_degrees=(4, 8), act="gelu_tanh", w_std=0.02, b_std=None),
+    # the same MLP with 8-bit (E4M3, per-row scale) weights, decode
+    "mlp70b_w8": MLPConfig("mlp70b_w8", hidden=8192, ffn=28672, tokens=(1, 16, 64),
+                           tp_degrees=(4, 8), act="gelu_tanh", w_std=0.02, b_std=None,
+                           weights="e4m3"),
     # Llama-3-70B-shaped attention projections, prefill
     "attn70b": AttnConfig("attn70b", hidden=8192, n_q_heads=64, n_kv_heads=8,
                           head_dim=128, tokens=(4096,), tp_degrees=(8,), w_std=0.02,
@@ -198,6 +210,23 @@ def attn_inputs(cfg: AttnConfig, T: int, seed: int = 0, with_bias: bool = False
     b_qkv = normal_bf16((nqkv,), 0.01, seed, IDX_QKV_B) if with_bias else None
     b_o = normal_bf16((H,), 0.01, seed, IDX_O_B) if with_bias else None
     return {"x": x, "w_qkv": w_qkv, "b_qkv": b_qkv, "ctx": ctx, "w_o": w_o, "b_o": b_o}
+
+
+def quantize_e4m3_rows(w: torch.Tensor, rows_per_chunk: int = 2048
+                       ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """8-bit storage of a [N, K] weight (recipe in the module docstring):
+    returns (q [N, K] uint8 E4M3 codes, scale [N] float32)."""
+    n = int(w.shape[0])
+    q = torch.empty(tuple(w.shape), dtype=torch.uint8)
+    scale = torch.empty(n, dtype=torch.float32)
+    for r0 in range(0, n, rows_per_chunk):
+        r1 = min(n, r0 + rows_per_chunk)
+        wf = w[r0:r1].to(torch.float32)
+        amax = wf.abs().amax(dim=1)
+        sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        q[r0:r1] = (wf / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        scale[r0:r1] = sc
+    return q, scale
 
 
 def sample_rows(T: int, count: int, seed: int = 0) -> List[int]:
