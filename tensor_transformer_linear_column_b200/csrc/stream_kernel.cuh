@@ -394,23 +394,33 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
     if constexpr (kW8) {
-      // ---------------- warps 0-3, first: E4M3 -> bf16.  Thread t rewrites row
-      // t of every box's weight tile, 8 elements (16 bytes) at a time, into the
-      // 128-byte-swizzled layout of a TMA tile (16-byte chunk j of row t at
-      // chunk j ^ (t % 8)), which the MMA descriptor expects.
+      // ---------------- warps 0-3, first: E4M3 -> bf16.  A pass converts 32
+      // rows of a box's 64-byte rows: thread t takes the 16 codes in chunk
+      // c = t % 4 of row t / 4, so each warp reads 512 contiguous bytes (no
+      // bank conflicts; a thread-per-row walk at a 64-byte stride puts 16 lanes
+      // on the same banks).  The 16 bf16 values are 16-byte chunks 2c and
+      // 2c + 1 of the row in the 128-byte-swizzled layout of a TMA tile (chunk
+      // j of row r at chunk j ^ (r % 8)), which the MMA descriptor expects.
       const int t = static_cast<int>(threadIdx.x);
+      const int c = t & 3;
       int s = 0;
       uint32_t ph = 0u;
       bool ok = true;
       for (int i = 0; i < nbox; ++i) {
         ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
         if (ok) {
-          const uint8_t* src = smem + s * p.stage_bytes + w8off + t * kStreamTileK;
-          uint8_t* dst = smem + s * p.stage_bytes + t * 128;
+          uint8_t* st = smem + s * p.stage_bytes;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint2 q = *reinterpret_cast<const uint2*>(src + j * 8);
-            *reinterpret_cast<uint4*>(dst + ((j ^ (t & 7)) * 16)) = e4m3x8_to_bf16x8(q);
+          for (int pass = 0; pass < kStreamTileM / 32; ++pass) {
+            const int r = pass * 32 + (t >> 2);
+            const uint4 q =
+                *reinterpret_cast<const uint4*>(st + w8off + r * kStreamTileK + c * 16);
+            uint8_t* dst = st + r * 128;
+            const int sw = r & 7;
+            *reinterpret_cast<uint4*>(dst + (((2 * c) ^ sw) * 16)) =
+                e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
+            *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ sw) * 16)) =
+                e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
           }
           fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
         }
