@@ -47,10 +47,11 @@
 //
 // 8-bit weights (kW8): the weight is FP8 E4M3 with one fp32 scale per row
 // (drpranayjha.com "AI Infrastructure series, Part 5", section "Reason 2":
-// decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 into a
-// staging buffer; the four epilogue warps, idle while the weights stream,
-// rewrite it as the bf16 tile the MMA reads (exact: every E4M3 value is a bf16
-// value), and the row scale multiplies the fp32 sum before bias and activation.
+// decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 into the
+// upper half of the stage's 16 KB weight tile; the four epilogue warps, idle
+// while the weights stream, rewrite it in place as the bf16 tile the MMA reads
+// (exact: every E4M3 value is a bf16 value), and the row scale multiplies the
+// fp32 sum before bias and activation.
 // The MMAs and everything after them are those of the bf16 kernel; HBM traffic
 // is halved.
 //
@@ -251,8 +252,9 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   const uint32_t x_bytes = static_cast<uint32_t>(p.t_pad) * kStreamTileK * 2;
   const uint32_t w_bytes = kStreamTileM * kStreamTileK * 2;  // one k-block of W: 16 KB
   const uint32_t xoff = static_cast<uint32_t>(kpb) * w_bytes;  // x tiles follow the W tiles
-  // 8-bit weights (kpb == 1): the E4M3 tile lands in staging after x
-  const uint32_t w8off = w_bytes + x_bytes;
+  // 8-bit weights (kpb == 1): the 8 KB E4M3 tile lands in the second half of
+  // the stage's bf16 weight tile and is converted in place
+  const uint32_t w8off = w_bytes - kStreamW8Bytes;
   const uint32_t wdst = kW8 ? w8off : 0u;
   const uint32_t tx_bytes =
       kW8 ? kStreamW8Bytes + x_bytes : static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
@@ -394,13 +396,18 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
     if constexpr (kW8) {
-      // ---------------- warps 0-3, first: E4M3 -> bf16.  A pass converts 32
-      // rows of a box's 64-byte rows: thread t takes the 16 codes in chunk
-      // c = t % 4 of row t / 4, so each warp reads 512 contiguous bytes (no
-      // bank conflicts; a thread-per-row walk at a 64-byte stride puts 16 lanes
-      // on the same banks).  The 16 bf16 values are 16-byte chunks 2c and
-      // 2c + 1 of the row in the 128-byte-swizzled layout of a TMA tile (chunk
-      // j of row r at chunk j ^ (r % 8)), which the MMA descriptor expects.
+      // ---------------- warps 0-3, first: E4M3 -> bf16, in place.  A box's
+      // 64-byte E4M3 rows occupy the upper half of the 16 KB tile whose 128-byte
+      // bf16 rows they become, so all 128 threads read their codes into
+      // registers before any thread writes (named barrier 1, reached by every
+      // converter thread once per box whatever its wait returned).  Thread t
+      // takes the 16 codes in chunk c = t % 4 of rows t / 4 + 32 pass: a warp
+      // reads 512 contiguous bytes per pass (no bank conflicts; a
+      // thread-per-row walk at a 64-byte stride puts 16 lanes on the same
+      // banks).  The 16 bf16 values are 16-byte chunks 2c and 2c + 1 of the
+      // row in the 128-byte-swizzled layout of a TMA tile (chunk j of row r at
+      // chunk j ^ (r % 8)), which the MMA descriptor expects.
+      constexpr int kPasses = kStreamTileM / 32;
       const int t = static_cast<int>(threadIdx.x);
       const int c = t & 3;
       int s = 0;
@@ -408,19 +415,25 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       bool ok = true;
       for (int i = 0; i < nbox; ++i) {
         ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
-        if (ok) {
-          uint8_t* st = smem + s * p.stage_bytes;
+        uint8_t* st = smem + s * p.stage_bytes;
+        uint4 q[kPasses];
 #pragma unroll
-          for (int pass = 0; pass < kStreamTileM / 32; ++pass) {
+        for (int pass = 0; pass < kPasses; ++pass) {
+          const int r = pass * 32 + (t >> 2);
+          q[pass] = ok ? *reinterpret_cast<const uint4*>(st + w8off + r * kStreamTileK + c * 16)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+        named_barrier_sync(1, 128);
+        if (ok) {
+#pragma unroll
+          for (int pass = 0; pass < kPasses; ++pass) {
             const int r = pass * 32 + (t >> 2);
-            const uint4 q =
-                *reinterpret_cast<const uint4*>(st + w8off + r * kStreamTileK + c * 16);
             uint8_t* dst = st + r * 128;
             const int sw = r & 7;
             *reinterpret_cast<uint4*>(dst + (((2 * c) ^ sw) * 16)) =
-                e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
+                e4m3x8_to_bf16x8(make_uint2(q[pass].x, q[pass].y));
             *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ sw) * 16)) =
-                e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
+                e4m3x8_to_bf16x8(make_uint2(q[pass].z, q[pass].w));
           }
           fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
         }

@@ -273,8 +273,8 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
         static_cast<long>(hi - lo) * tpb::kStreamTileM * tpb::kStreamTileK * (w8 ? 1 : 2);
     const int budget = (w_cta >= 256 * 1024 ? 110 : 72) * 1024 -
                        tpb::stream_recv_bytes(p.T, p.csize);
-    // one k-block of W (bf16) and x, plus its 8 KB staging tile for 8-bit W
-    const int kb_bytes = p.stage_bytes + (w8 ? tpb::kStreamW8Bytes : 0);
+    // one k-block of W (bf16) and x; an 8-bit tile is converted in place
+    const int kb_bytes = p.stage_bytes;
     bool even = p.spc == 1;
     for (int r = 0; even && r < p.csize; ++r) {
       tpb::stream_cta_range(p, r, lo, hi);
