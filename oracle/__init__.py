@@ -22,3 +22,4 @@ from .tp_oracle import (  # noqa: F401
     shard_sum,
     to_f64,
 )
+from .tp_backward import act_grad, gelu_tanh_grad, mlp_block_backward  # noqa: F401
