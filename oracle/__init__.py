@@ -22,4 +22,5 @@ from .tp_oracle import (  # noqa: F401
     shard_sum,
     to_f64,
 )
+from .tp_attention import attend_head, attn_core, empty_cache  # noqa: F401
 from .tp_backward import act_grad, gelu_tanh_grad, mlp_block_backward  # noqa: F401
