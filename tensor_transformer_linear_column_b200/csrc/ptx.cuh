@@ -442,13 +442,13 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 q) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Order this thread's generic-proxy shared-memory writes before later
-// async-proxy reads of them (tcgen05.mma operands, bulk copies).
 // Barrier `id` (1-15) among `nthreads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (tcgen05.mma operands, bulk copies).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
