@@ -225,7 +225,9 @@ tp_status tp_mlp_forward_noalloc(const tp_bf16* x, const tp_bf16* w1, const tp_b
  * tp_rowpar_gemm_reduce and tp_mlp_forward.  These calls always use the
  * weight-streaming kernel: T <= 128 (else TP_ERR_UNSUPPORTED); row-parallel
  * calls whose shards would not fit two per streaming CTA also return
- * TP_ERR_UNSUPPORTED (none of t <= 8 at the 70B shapes).
+ * TP_ERR_UNSUPPORTED (none of t <= 8 at the 70B shapes).  tp_mlp_forward_w8
+ * checks both layers' splits before it launches anything, so such a return
+ * leaves the workspace and out untouched.
  */
 tp_status tp_colpar_gemm_gelu_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,
                                  const tp_bf16* b, int T, int K, int N, int tp_degree, int act,

@@ -460,6 +460,15 @@ tp_status run_rowpar(const tp_bf16* h, const tp_bf16* w, const tp_bf16* b, int T
   return launch_tiled(*dev, h, w, b, T, K, N, t, 0, out, stream);
 }
 
+// Geometry of an 8-bit streaming launch: csize == 0 when the split is not
+// supported (no cluster shape, or more than two shards per CTA).
+StreamGeometry w8_geometry(const DeviceInfo& dev, int T, int K, int N, int shards) {
+  const int t_pad = (T + 15) / 16 * 16;
+  StreamGeometry g = stream_geometry(N, K / 64, shards, t_pad, dev.sms);
+  if (g.spc > 2) g.csize = 0;
+  return g;
+}
+
 // 8-bit weights: the streaming kernel only (T <= kStreamMaxTokens).
 tp_status run_linear_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,
                         const tp_bf16* b, int T, int K, int N, int shards, int act, tp_bf16* out,
@@ -467,8 +476,7 @@ tp_status run_linear_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scal
   if (T > kStreamMaxTokens) return TP_ERR_UNSUPPORTED;
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  const int t_pad = (T + 15) / 16 * 16;
-  const StreamGeometry g = stream_geometry(N, K / 64, shards, t_pad, dev->sms);
+  const StreamGeometry g = w8_geometry(*dev, T, K, N, shards);
   if (g.csize == 0) return TP_ERR_UNSUPPORTED;
   return launch_stream(*dev, g, x, w8, w_scale, b, T, K, N, shards, act, out, stream);
 }
@@ -599,6 +607,12 @@ tp_status tp_mlp_forward_w8(const tp_bf16* x, const uint8_t* w1, const float* s1
   if (workspace == nullptr || workspace_bytes < tp_mlp_workspace_bytes(T, F))
     return TP_ERR_WORKSPACE;
   if (!aligned16(workspace)) return TP_ERR_ALIGN;
+  // both layers' splits are checked before the first launch, so an
+  // unsupported split leaves the workspace untouched
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  if (w8_geometry(*dev, T, H, F, 1).csize == 0 || w8_geometry(*dev, T, F, H, tp_degree).csize == 0)
+    return TP_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   tp_bf16* h = static_cast<tp_bf16*>(workspace);
   tp_status s = run_linear_w8(x, w1, s1, b1, T, H, F, 1, act, h, st);

@@ -71,6 +71,25 @@ def test_w8_rowpar_more_than_two_shards_per_cta_is_unsupported():
     assert e.value.status == tp.TP_ERR_UNSUPPORTED
 
 
+def test_w8_mlp_unsupported_split_launches_nothing():
+    # t = 3 over F = 576: the second layer would need three shards per CTA;
+    # the call must refuse before its first layer writes the workspace
+    dev = _dev()
+    T, H, F = 5, 256, 576
+    x = workloads.random_bf16_small((T, H), 1.0, 7700).to(dev)
+    q1, s1 = _w8((F, H), 0.05, 7701)
+    q2, s2 = _w8((H, F), 0.05, 7702)
+    ws = torch.full((tp.tp_mlp_workspace_bytes(T, F),), 0x5A, dtype=torch.uint8, device=dev)
+    out = torch.full((T, H), 7.0, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_mlp_forward_w8(x, q1.to(dev), s1.to(dev), None, q2.to(dev), s2.to(dev), None, 3,
+                             "gelu_tanh", out=out, workspace=ws)
+    assert e.value.status == tp.TP_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert bool((ws == 0x5A).all())
+    assert bool((out == 7.0).all())
+
+
 @pytest.fixture(scope="module")
 def mlp70b_w8():
     cfg = workloads.CONFIGS["mlp70b_w8"]
