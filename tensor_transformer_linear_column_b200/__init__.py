@@ -125,9 +125,25 @@ def _ptr_typed(t: Optional[torch.Tensor], name: str, dev: torch.device,
     return t.data_ptr()
 
 
+def _device(t: torch.Tensor) -> torch.device:
+    """The device of a call: that of its first tensor, which must be the current
+    CUDA device (the library launches there; a host or other-device pointer
+    handed to a kernel would fault)."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"inputs are on {t.device} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({t.device.index})")
+    return t.device
+
+
 def _stream(stream: Optional[torch.cuda.Stream]) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if stream.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {stream.device}, not the current device")
+    return stream.cuda_stream
 
 
 def _check(status: int, where: str) -> None:
@@ -147,9 +163,9 @@ def tp_colpar_gemm_gelu(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tens
     N = w.shape[0]
     if w.shape[1] != K:
         raise ValueError("w must be [N, K]")
+    dev = _device(x)
     if out is None:
-        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
-    dev = x.device
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
     st = load().tp_colpar_gemm_gelu(_ptr(x, "x", dev), _ptr(w, "w", dev), _ptr(b, "b", dev),
                                     T, K, N, int(tp_degree), _act(act), _ptr(out, "out", dev),
                                     _stream(stream))
@@ -165,9 +181,9 @@ def tp_rowpar_gemm_reduce(h: torch.Tensor, w: torch.Tensor, b: Optional[torch.Te
     N = w.shape[0]
     if w.shape[1] != K:
         raise ValueError("w must be [N, K]")
+    dev = _device(h)
     if out is None:
-        out = torch.empty((T, N), dtype=torch.bfloat16, device=h.device)
-    dev = h.device
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
     st = load().tp_rowpar_gemm_reduce(_ptr(h, "h", dev), _ptr(w, "w", dev), _ptr(b, "b", dev),
                                       T, K, N, int(tp_degree), _ptr(out, "out", dev),
                                       _stream(stream))
@@ -189,7 +205,7 @@ def tp_mlp_forward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor]
     F = w1.shape[0]
     if w1.shape[1] != H or tuple(w2.shape) != (H, F):
         raise ValueError("w1 must be [F, H] and w2 [H, F]")
-    dev = x.device
+    dev = _device(x)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     need = tp_mlp_workspace_bytes(T, F)
@@ -216,7 +232,7 @@ def tp_colpar_gemm_gelu_w8(x: torch.Tensor, w8: torch.Tensor, w_scale: torch.Ten
     N = w8.shape[0]
     if w8.shape[1] != K or tuple(w_scale.shape) != (N,):
         raise ValueError("w8 must be [N, K] and w_scale [N]")
-    dev = x.device
+    dev = _device(x)
     if out is None:
         out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
     st = load().tp_colpar_gemm_gelu_w8(
@@ -236,7 +252,7 @@ def tp_rowpar_gemm_reduce_w8(h: torch.Tensor, w8: torch.Tensor, w_scale: torch.T
     N = w8.shape[0]
     if w8.shape[1] != K or tuple(w_scale.shape) != (N,):
         raise ValueError("w8 must be [N, K] and w_scale [N]")
-    dev = h.device
+    dev = _device(h)
     if out is None:
         out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
     st = load().tp_rowpar_gemm_reduce_w8(
@@ -261,7 +277,7 @@ def tp_mlp_forward_w8(x: torch.Tensor, w1: torch.Tensor, s1: torch.Tensor,
         raise ValueError("w1 must be [F, H] and w2 [H, F]")
     if tuple(s1.shape) != (F,) or tuple(s2.shape) != (H,):
         raise ValueError("s1 must be [F] and s2 [H]")
-    dev = x.device
+    dev = _device(x)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     need = tp_mlp_workspace_bytes(T, F)
@@ -294,7 +310,7 @@ def tp_mlp_forward_noalloc(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch
     F = w1.shape[0]
     if w1.shape[1] != H or tuple(w2.shape) != (H, F):
         raise ValueError("w1 must be [F, H] and w2 [H, F]")
-    dev = x.device
+    dev = _device(x)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     st = load().tp_mlp_forward_noalloc(_ptr(x, "x", dev), _ptr(w1, "w1", dev),
@@ -313,7 +329,7 @@ def tp_attn_proj_forward(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: Optional[t
                          stream: Optional[torch.cuda.Stream] = None):
     """(qkv, y): the head-split QKV projection and the row-parallel output projection."""
     T, H = x.shape
-    dev = x.device
+    dev = _device(x)
     nqkv = (n_q_heads + 2 * n_kv_heads) * head_dim
     if qkv_out is None:
         qkv_out = torch.empty((T, nqkv), dtype=torch.bfloat16, device=dev)

@@ -186,12 +186,31 @@ def test_decode_threshold_setting(lib):
         tp.tp_set_decode_max_tokens(prev)
 
 
-def test_python_binding_type_checks():
+def test_python_binding_rejects_host_tensors():
+    # host pointers handed to a kernel would fault: every wrapper refuses
+    # non-CUDA inputs before it reaches the library
     import torch
-    x = torch.zeros(8, 256, dtype=torch.float32)
-    w = torch.zeros(1024, 256, dtype=torch.bfloat16)
-    with pytest.raises(TypeError):
-        tp.tp_colpar_gemm_gelu(x, w, None, 2)
+    bf = torch.bfloat16
+    x = torch.zeros(8, 256, dtype=bf)
+    w1, w2 = torch.zeros(1024, 256, dtype=bf), torch.zeros(256, 1024, dtype=bf)
+    q1, q2 = torch.zeros(1024, 256, dtype=torch.uint8), torch.zeros(256, 1024, dtype=torch.uint8)
+    s1, s2 = torch.ones(1024), torch.ones(256)
+    h = torch.zeros(8, 1024, dtype=bf)
+    calls = [
+        lambda: tp.tp_colpar_gemm_gelu(x, w1, None, 2),
+        lambda: tp.tp_rowpar_gemm_reduce(h, w2, None, 2),
+        lambda: tp.tp_mlp_forward(x, w1, None, w2, None, 2),
+        lambda: tp.tp_mlp_forward_noalloc(x, w1, None, w2, None, 2),
+        lambda: tp.tp_colpar_gemm_gelu_w8(x, q1, s1, None, 2),
+        lambda: tp.tp_rowpar_gemm_reduce_w8(h, q2, s2, None, 2),
+        lambda: tp.tp_mlp_forward_w8(x, q1, s1, None, q2, s2, None, 2),
+        lambda: tp.tp_attn_proj_forward(x, torch.zeros(384, 256, dtype=bf), None,
+                                        torch.zeros(8, 256, dtype=bf),
+                                        torch.zeros(256, 256, dtype=bf), None, 4, 1, 64, 1),
+    ]
+    for c in calls:
+        with pytest.raises(ValueError, match="CUDA tensors"):
+            c()
 
 
 def test_launch_options_setting(lib):

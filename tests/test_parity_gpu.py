@@ -406,3 +406,17 @@ def test_graph_replayed_decode_step_matches_eager(sq_weights):
     for T in xs:
         assert torch.equal(outs[T], eager[T])
     assert_parity(outs[64], oracle.colpar_linear(xs[64].cpu(), w, None, 2, "none"), "graph T=64")
+
+
+def test_binding_checks_dtype_and_device_before_the_library():
+    # no launch happens in any of these: the binding refuses first
+    dev = _dev()
+    x = torch.zeros(8, 256, dtype=torch.float32, device=dev)
+    w = torch.zeros(1024, 256, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(TypeError):
+        tp.tp_colpar_gemm_gelu(x, w, None, 2)
+    xb = x.to(torch.bfloat16)
+    with pytest.raises(ValueError):
+        tp.tp_colpar_gemm_gelu(xb, w.cpu(), None, 2)
+    with pytest.raises(ValueError):
+        tp.tp_colpar_gemm_gelu(xb.cpu(), w, None, 2)
