@@ -292,6 +292,36 @@ int tp_get_decode_max_tokens(void);
 tp_status tp_set_launch_options(unsigned int flags);
 unsigned int tp_get_launch_options(void);
 
+/*
+ * The launch the weight-streaming kernel makes for one linear layer, computed
+ * for a device with `sms` multiprocessors and `max_smem` bytes of opt-in
+ * shared memory per block.  Host arithmetic only: no device is touched, so it
+ * also runs without a GPU.
+ *   T, K, N     tokens, input features, output features of the layer
+ *   row_shards  1 for a column-parallel layer, t for a row-parallel one
+ *               (t must divide K into multiples of 64)
+ *   w8          nonzero for 8-bit weights (the *_w8 calls)
+ * Fills *plan and returns TP_OK; TP_ERR_UNSUPPORTED when the streaming kernel
+ * does not take the layer (T > 128, no cluster shape, or an 8-bit split with
+ * more than two shards per CTA: the bf16 calls then use the tiled kernel, the
+ * *_w8 calls return TP_ERR_UNSUPPORTED); TP_ERR_NULL for a NULL plan;
+ * TP_ERR_SHAPE or TP_ERR_TP_DEGREE for bad sizes.  Whether a bf16 call
+ * streams at all also depends on tp_set_decode_max_tokens.
+ */
+typedef struct {
+  int grid_x;           /* 128-row weight tiles (the grid is grid_x x cluster CTAs) */
+  int cluster;          /* CTAs per thread-block cluster, splitting K */
+  int jsplit;           /* CTAs that share one shard's K-slice */
+  int shards_per_cta;   /* row-parallel shards one CTA sums */
+  int stages;           /* depth of the shared-memory ring */
+  int kblocks_per_box;  /* 64-column k-blocks per TMA box */
+  int stage_bytes;      /* bytes of one ring stage */
+  int smem_bytes;       /* dynamic shared memory per CTA */
+  int l2_ahead;         /* boxes sent to L2 before the wait on the preceding grid */
+} tp_stream_plan_t;
+tp_status tp_stream_plan(int T, int K, int N, int row_shards, int w8, int sms, int max_smem,
+                         tp_stream_plan_t* plan);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

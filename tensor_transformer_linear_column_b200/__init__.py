@@ -55,7 +55,20 @@ SIGNATURES = {
     "tp_get_decode_max_tokens": (_I, []),
     "tp_set_launch_options": (_I, [ctypes.c_uint]),
     "tp_get_launch_options": (ctypes.c_uint, []),
+    "tp_stream_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _P]),
 }
+
+
+class StreamPlan(ctypes.Structure):
+    """tp_stream_plan_t of include/tp_block.h."""
+    _fields_ = [(name, ctypes.c_int) for name in (
+        "grid_x", "cluster", "jsplit", "shards_per_cta", "stages", "kblocks_per_box",
+        "stage_bytes", "smem_bytes", "l2_ahead")]
+
+
+# a B200: 148 multiprocessors, 227 KB of opt-in shared memory per block
+B200_SMS = 148
+B200_MAX_SMEM = 232448
 
 
 class TPError(RuntimeError):
@@ -356,6 +369,17 @@ def tp_set_decode_max_tokens(max_tokens: int) -> None:
 
 def tp_get_decode_max_tokens() -> int:
     return int(load().tp_get_decode_max_tokens())
+
+
+def tp_stream_plan(T: int, K: int, N: int, row_shards: int = 1, w8: bool = False,
+                   sms: int = B200_SMS, max_smem: int = B200_MAX_SMEM) -> dict:
+    """The weight-streaming kernel's launch for one layer (host arithmetic, no GPU
+    needed); raises TPError (e.g. TP_ERR_UNSUPPORTED) when it would not stream."""
+    plan = StreamPlan()
+    st = load().tp_stream_plan(int(T), int(K), int(N), int(row_shards), 1 if w8 else 0,
+                               int(sms), int(max_smem), ctypes.addressof(plan))
+    _check(st, "tp_stream_plan")
+    return {name: getattr(plan, name) for name, _ in StreamPlan._fields_}
 
 
 def tp_set_launch_options(flags: int) -> None:

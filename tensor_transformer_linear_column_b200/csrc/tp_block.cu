@@ -237,17 +237,13 @@ StreamGeometry stream_geometry(int N, int kb_total, int shards, int t_pad, int s
   return fallback;
 }
 
-// Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
-// sum (1 for the column-parallel layer).  Requires T <= 128 and a geometry
-// from stream_geometry().  With `w_scale` non-null the weight is 8-bit (E4M3
-// bytes, [N, K]) and w_scale[n] scales row n; the geometry must then keep
-// spc <= 2 (both shard regions are drained after all tiles are converted).
-tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const tp_bf16* x,
-                        const void* w, const float* w_scale, const tp_bf16* b, int T, int K,
-                        int N, int shards, int act, tp_bf16* out, cudaStream_t stream) {
-  const bool w8 = w_scale != nullptr;
-  if (w8 && geo.spc > 2) return TP_ERR_UNSUPPORTED;
-  StreamParams p{};
+// The sizes of a streaming launch (everything but pointers and options):
+// geometry, ring depth, box size, shared memory.  Host arithmetic only; the
+// device enters through max_smem.  TP_ERR_UNSUPPORTED if it does not fit.
+tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, int K, int N,
+                      int shards, StreamParams& p, int& smem) {
+  if (geo.csize == 0 || (w8 && geo.spc > 2)) return TP_ERR_UNSUPPORTED;
+  p = StreamParams{};
   p.T = T;
   p.K = K;
   p.N = N;
@@ -292,18 +288,33 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
     // on their own
     p.l2_ahead = w_cta >= 256 * 1024 ? 0 : 2;
   }
+  // large T: the receive buffer leaves room for two stages only
+  while (p.stages > 2 &&
+         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize) > max_smem)
+    --p.stages;
+  smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize);
+  return smem > max_smem ? TP_ERR_UNSUPPORTED : TP_OK;
+}
+
+// Weight-streaming kernel.  `shards` groups the reduction for the row-parallel
+// sum (1 for the column-parallel layer).  Requires T <= 128 and a geometry
+// from stream_geometry().  With `w_scale` non-null the weight is 8-bit (E4M3
+// bytes, [N, K]) and w_scale[n] scales row n; the geometry must then keep
+// spc <= 2 (both shard regions are drained after all tiles are converted).
+tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const tp_bf16* x,
+                        const void* w, const float* w_scale, const tp_bf16* b, int T, int K,
+                        int N, int shards, int act, tp_bf16* out, cudaStream_t stream) {
+  const bool w8 = w_scale != nullptr;
+  StreamParams p;
+  int smem = 0;
+  const tp_status planned = plan_stream(dev.max_smem, geo, w8, T, K, N, shards, p, smem);
+  if (planned != TP_OK) return planned;
   p.act = act;
   p.prefetch_w = prefetch_weights();
   p.bias = b;
   p.w_scale = w_scale;
   p.out = out;
   const int n_tiles = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
-  // large T: the receive buffer leaves room for two stages only
-  while (p.stages > 2 &&
-         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize) > dev.max_smem)
-    --p.stages;
-  const int smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize);
-  if (smem > dev.max_smem) return TP_ERR_UNSUPPORTED;
 
   CUtensorMap tw, tx;
   const bool tw_ok =
@@ -618,6 +629,31 @@ tp_status tp_mlp_forward_w8(const tp_bf16* x, const uint8_t* w1, const float* s1
   tp_status s = run_linear_w8(x, w1, s1, b1, T, H, F, 1, act, h, st);
   if (s != TP_OK) return s;
   return run_linear_w8(h, w2, s2, b2, T, F, H, tp_degree, TP_ACT_NONE, out, st);
+}
+
+tp_status tp_stream_plan(int T, int K, int N, int row_shards, int w8, int sms, int max_smem,
+                         tp_stream_plan_t* plan) {
+  if (plan == nullptr) return TP_ERR_NULL;
+  if (T < 1 || !feat_ok(K) || !feat_ok(N) || sms < 1 || max_smem < 1) return TP_ERR_SHAPE;
+  if (row_shards < 1 || K % row_shards != 0 || (K / row_shards) % 64 != 0)
+    return TP_ERR_TP_DEGREE;
+  if (T > kStreamMaxTokens) return TP_ERR_UNSUPPORTED;
+  const int t_pad = (T + 15) / 16 * 16;
+  const StreamGeometry g = stream_geometry(N, K / 64, row_shards, t_pad, sms);
+  StreamParams p;
+  int smem = 0;
+  const tp_status s = plan_stream(max_smem, g, w8 != 0, T, K, N, row_shards, p, smem);
+  if (s != TP_OK) return s;
+  plan->grid_x = (N + tpb::kStreamTileM - 1) / tpb::kStreamTileM;
+  plan->cluster = p.csize;
+  plan->jsplit = p.jsplit;
+  plan->shards_per_cta = p.spc;
+  plan->stages = p.stages;
+  plan->kblocks_per_box = p.kpb;
+  plan->stage_bytes = p.stage_bytes;
+  plan->smem_bytes = smem;
+  plan->l2_ahead = p.l2_ahead;
+  return TP_OK;
 }
 
 const char* tp_status_string(tp_status status) {

@@ -225,3 +225,95 @@ def test_launch_options_setting(lib):
         assert tp.tp_get_launch_options() == 0
     finally:
         tp.tp_set_launch_options(prev)
+
+
+# ---------------------------------------------------------------- launch plans (host only)
+
+def _profile_row(path, metric):
+    """The three per-launch values of `metric` in a committed ncu summary table."""
+    with open(path) as f:
+        for line in f:
+            if line.startswith(f"| `{metric}` |"):
+                cells = [c.strip() for c in line.strip().strip("|").split("|")[1:]]
+                return [float(c.split()[0]) for c in cells]
+    raise AssertionError(f"{metric} not in {path}")
+
+
+def test_stream_plan_matches_the_profiled_sq4096_launches():
+    # the committed ncu capture of the 4096 x 4096 decode step (T = 1, 8, 64)
+    # records what the GPU launched; the host plan must still produce it
+    path = os.path.join(ROOT, "profiles", "stream_gemm_kernel_sq4096.md")
+    smem_kb = _profile_row(path, "launch__shared_mem_per_block_dynamic")
+    grid = _profile_row(path, "launch__grid_size")
+    cluster = _profile_row(path, "launch__cluster_dim_y")
+    for i, T in enumerate((1, 8, 64)):
+        p = tp.tp_stream_plan(T, 4096, 4096)
+        assert p["smem_bytes"] == round(smem_kb[i] * 1000)
+        assert p["grid_x"] * p["cluster"] == grid[i]
+        assert p["cluster"] == cluster[i]
+
+
+def test_stream_plan_ring_depths_of_the_70b_decode():
+    # 8-bit tiles are converted in place, so a stage holds one bf16 tile + x
+    for T, stages in ((1, 6), (16, 6), (64, 4)):
+        p = tp.tp_stream_plan(T, 8192, 28672, 1, w8=True)
+        assert p["stages"] == stages and p["kblocks_per_box"] == 1
+        t_pad = (T + 15) // 16 * 16
+        assert p["stage_bytes"] == (128 + t_pad) * 64 * 2
+    # bf16 up-projection at T = 1: two k-blocks per box, three boxes in flight
+    p = tp.tp_stream_plan(1, 8192, 28672)
+    assert p["kblocks_per_box"] == 2 and p["stages"] == 3
+
+
+@pytest.mark.parametrize("w8", [False, True])
+def test_stream_plan_invariants(w8):
+    sms, max_smem = tp.B200_SMS, tp.B200_MAX_SMEM
+    checked = 0
+    for T in (1, 2, 15, 16, 17, 33, 64, 65, 100, 128):
+        for K, N in ((64, 64), (256, 1088), (4096, 4096), (8192, 28672), (28672, 8192),
+                     (16384, 192), (576, 320)):
+            for shards in (1, 2, 3, 4, 8, 16):
+                if K % shards or (K // shards) % 64:
+                    continue
+                try:
+                    p = tp.tp_stream_plan(T, K, N, shards, w8)
+                except tp.TPError as e:
+                    assert e.status == tp.TP_ERR_UNSUPPORTED
+                    continue
+                checked += 1
+                t_pad = (T + 15) // 16 * 16
+                assert p["grid_x"] == (N + 127) // 128
+                assert p["cluster"] in (1, 2, 4, 8)
+                if p["cluster"] >= shards:
+                    assert p["jsplit"] * shards == p["cluster"] and p["shards_per_cta"] == 1
+                else:
+                    assert p["jsplit"] == 1 and p["shards_per_cta"] * p["cluster"] == shards
+                    assert t_pad <= 64  # the running sum of several shards lives in registers
+                assert 2 <= p["stages"] <= 8
+                assert p["kblocks_per_box"] in (1, 2)
+                assert p["stage_bytes"] == p["kblocks_per_box"] * (128 + t_pad) * 128
+                assert p["smem_bytes"] <= max_smem
+                assert p["smem_bytes"] >= p["stages"] * p["stage_bytes"]
+                if w8:
+                    assert p["kblocks_per_box"] == 1 and p["shards_per_cta"] <= 2
+                # every CTA resident at once whenever some cluster shape allows it
+                if p["grid_x"] * p["cluster"] > 2 * sms:
+                    assert p["cluster"] == 1 or shards > 1
+    assert checked > 100
+
+
+def test_stream_plan_errors(lib):
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_stream_plan(129, 4096, 4096)
+    assert e.value.status == tp.TP_ERR_UNSUPPORTED
+    with pytest.raises(tp.TPError) as e:  # 8-bit: three shards would share one CTA
+        tp.tp_stream_plan(5, 576, 256, 3, w8=True)
+    assert e.value.status == tp.TP_ERR_UNSUPPORTED
+    assert tp.tp_stream_plan(5, 576, 256, 3)["shards_per_cta"] == 3  # bf16 takes it
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_stream_plan(8, 4096, 4096, 3)
+    assert e.value.status == tp.TP_ERR_TP_DEGREE
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_stream_plan(8, 100, 4096)
+    assert e.value.status == tp.TP_ERR_SHAPE
+    assert lib.tp_stream_plan(8, 4096, 4096, 1, 0, 148, 232448, None) == tp.TP_ERR_NULL
