@@ -100,7 +100,8 @@ constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when sp
 // Shared memory layout (dynamic, base rounded up to 1024 B):
 //   [0, stages * stage_bytes)   pipeline: per stage kpb W tiles (16 KB each) then kpb x
 //                               tiles (t_pad * 128 B each); with 8-bit weights (kpb = 1)
-//                               then the 8 KB E4M3 staging tile [128][64] bytes
+//                               the 8 KB E4M3 tile [128][64] bytes lands in the upper
+//                               half of the W tile and is converted in place
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
 //   conv[stages] (8-bit weights: tile converted), tmem slot, abort flag
