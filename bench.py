@@ -4,11 +4,15 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload sq4096|tiny|mlp70b|mlp70b_w8|attn70b|mlp405b] [--tp T]
 
-Default workload: the pages' TP=2 square projection (W[4096, 4096] split by
-columns into 2 shards), decode batches T = 1, 8 and 64.  One step = one pass of
-the block's path over one batch of each T (3 column-parallel calls, 73 tokens).
-The other workloads are available for measurement with --workload
-(mlp70b_w8: the 70B-shaped MLP with 8-bit E4M3 weights and per-row scales).
+Default workload: the largest block of the measured set, the 405B-shaped MLP
+in prefill (x[8192, 16384], W1 [53248, 16384] split by columns into t = 8
+shards, GeLU, W2 [16384, 53248] split by rows with the fused 8-shard sum).  One
+step = one pass of the whole block over one batch: the column-parallel GEMM and
+the row-parallel GEMM with its on-chip all-reduce, 8192 tokens.  The other
+workloads are available with --workload: sq4096 (the pages' TP=2 square
+projection at decode batches T = 1, 8, 64), mlp70b (the 70B-shaped MLP decode),
+mlp70b_w8 (the same with 8-bit E4M3 weights and per-row scales), attn70b (the
+70B-shaped attention projections in prefill) and tiny.
 
 Timing: W warm-up steps, then exactly K steps captured in CUDA graphs and
 bracketed by a barrier + synchronize on both sides, timed with CUDA events on
@@ -53,6 +57,9 @@ KERNEL_SOURCES = {
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# default (timed steps, warm-up steps) per workload: about a second of timed work
+DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "mlp70b": (2000, 50),
+                 "mlp70b_w8": (2000, 50), "sq4096": (20000, 200), "tiny": (20000, 200)}
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -248,9 +255,9 @@ class Workload:
         self.outs = {T: torch.empty((T, self.hidden_out), dtype=torch.bfloat16, device=device)
                      for T in self.Ts}
         # rotate weight copies so each step reads weights evicted from L2
-        self.rot = 1
-        if rotate and self.weight_bytes < 4 * L2_BYTES:
-            self.rot = int(math.ceil(4 * L2_BYTES / self.weight_bytes))
+        assert self.weight_bytes == workload_weight_bytes(name)
+        self.rot = rotation_copies(self.weight_bytes) if rotate else 1
+        if self.rot > 1:
             base = self.weights[0]
             for _ in range(self.rot - 1):
                 if isinstance(base, tuple):
@@ -435,7 +442,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(name, runner.t, None),
+        "data": "synthetic", "config": workload_config(name, runner.t, args.options),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -444,7 +451,27 @@ def run_reference(args, world, rank):
     return 0
 
 
-def workload_config(name, t, wl):
+def workload_weight_bytes(name):
+    """Bytes of the weights one step reads per call (same count as Workload)."""
+    cfg = workloads.CONFIGS[name]
+    if name == "sq4096":
+        return cfg.k * cfg.n * 2
+    if name == "attn70b":
+        nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+        return (nqkv + cfg.n_q_heads * cfg.head_dim) * cfg.hidden * 2
+    if name == "mlp70b_w8":
+        return 2 * cfg.hidden * cfg.ffn + 4 * (cfg.hidden + cfg.ffn)
+    return 2 * cfg.hidden * cfg.ffn * 2
+
+
+def rotation_copies(weight_bytes):
+    """Weight copies rotated per call so each call reads weights evicted from L2."""
+    if weight_bytes < 4 * L2_BYTES:
+        return int(math.ceil(4 * L2_BYTES / weight_bytes))
+    return 1
+
+
+def workload_config(name, t, options):
     cfg = workloads.CONFIGS[name]
     desc = {
         "sq4096": "column-parallel projection W[4096,4096] bf16, t=2 column shards, decode T=1,8,64",
@@ -454,17 +481,17 @@ def workload_config(name, t, wl):
                      "8-bit weights (FP8 E4M3 codes, one fp32 scale per row)",
         "attn70b": "Llama-3-70B-shaped attention projections prefill T=4096, QKV 8192->10240 "
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
-        "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192",
+        "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192, column-parallel "
+                   "up-projection + row-parallel down-projection with the fused 8-shard sum",
     }[name]
-    c = {"workload": desc, "name": name, "tp_degree": t, "tokens": list(cfg.tokens),
-         "parallelism": "replicas (per-GPU block, t logical shards on chip)"}
-    if wl is not None:
-        c["l2"] = (f"weights rotated per call over {wl.rot} copies "
-                   f"({wl.rot * wl.weight_bytes / 1e6:.0f} MB >= 4x the 126 MB L2): every call "
-                   f"reads cold weights"
-                   if wl.rot > 1 else
-                   f"weights {wl.weight_bytes / 1e6:.0f} MB > 126 MB L2, read once per step")
-    return c
+    wb = workload_weight_bytes(name)
+    rot = rotation_copies(wb)
+    return {"workload": desc, "name": name, "tp_degree": t, "tokens": list(cfg.tokens),
+            "parallelism": "replicas (per-GPU block, t logical shards on chip)",
+            "l2": (f"weights rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
+                   f"the 126 MB L2): every call reads cold weights" if rot > 1 else
+                   f"weights {wb / 1e6:.0f} MB > 126 MB L2, read once per step"),
+            "launch_options": options}
 
 
 def run_ours(args, world, rank, local):
@@ -561,8 +588,7 @@ def run_ours(args, world, rank, local):
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0, sigma) bf16 inputs of the workload's shapes)",
-            "config": dict(workload_config(args.workload, wl.t, wl),
-                           launch_options=args.options),
+            "config": workload_config(args.workload, wl.t, args.options),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": wl.launches_per_step * K,
             "clocks": clocks,
@@ -686,10 +712,11 @@ def end_to_end(wl, stream, steps, world, dev):
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about a second of work for the workload)")
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="sq4096", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--workload", default="mlp405b", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--tp", type=int, default=None, help="tp degree (default: the workload's)")
     ap.add_argument("--options", choices=sorted(LAUNCH_OPTIONS), default="pdl+static_weights",
                     help="library launch options: the workload's weights are loaded once and "
@@ -699,6 +726,11 @@ def parse(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     args = ap.parse_args(argv)
+    steps, warmup = DEFAULT_STEPS.get(args.workload, (200, 10))
+    if args.steps is None:
+        args.steps = steps
+    if args.warmup is None:
+        args.warmup = warmup
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.steps < 1:

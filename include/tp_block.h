@@ -262,6 +262,24 @@ const char* tp_last_cuda_error(void);
 tp_status tp_device_error_check(void);
 
 /*
+ * Diagnostic (not part of the block): makes the library's bounded wait run out
+ * on purpose, so a caller or a test can check the timeout path without a fault
+ * or a hang.  Launches one CTA on `stream` in which two roles wait on barriers
+ * that nothing arrives on: the first with a limit of `limit_us` microseconds,
+ * the second with the library's normal limit (about one second) but sharing
+ * the CTA's abort flag, so it must give up as soon as the first one has.
+ *   limit_us  1 .. 1000000
+ *   result    device int[3], 16-byte aligned (written): what the two waits
+ *             returned (1 = completed, 0 = gave up; both are 0), and the
+ *             nanoseconds the second wait took
+ * After the kernel, tp_device_error_check() returns TP_ERR_DEVICE_TIMEOUT once
+ * and clears the error word.  Returns TP_ERR_NULL, TP_ERR_ALIGN or
+ * TP_ERR_UNSUPPORTED (limit out of range) before any launch, TP_ERR_CUDA if
+ * the launch fails.
+ */
+tp_status tp_diag_bounded_wait(unsigned int limit_us, int* result, tp_stream_t stream);
+
+/*
  * Token count at or below which a call takes the weight-streaming (decode)
  * kernels instead of the tiled (prefill) kernels.  `max_tokens` in [0, 128];
  * 0 sends every call to the tiled kernels.  Process-wide; returns

@@ -51,6 +51,7 @@ SIGNATURES = {
     "tp_status_string": (ctypes.c_char_p, [_I]),
     "tp_last_cuda_error": (ctypes.c_char_p, []),
     "tp_device_error_check": (_I, []),
+    "tp_diag_bounded_wait": (_I, [ctypes.c_uint, _P, _P]),
     "tp_set_decode_max_tokens": (_I, [_I]),
     "tp_get_decode_max_tokens": (_I, []),
     "tp_set_launch_options": (_I, [ctypes.c_uint]),
@@ -361,6 +362,19 @@ def tp_attn_proj_forward(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: Optional[t
 def tp_device_error_check() -> int:
     """Synchronise, then read and clear the kernels' device-side error word."""
     return int(load().tp_device_error_check())
+
+
+def tp_diag_bounded_wait(limit_us: int, result: torch.Tensor,
+                         stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Diagnostic: a kernel whose bounded waits run out on purpose (result: int32[3]
+    on the current device; see include/tp_block.h)."""
+    dev = _device(result)
+    if result.dtype != torch.int32 or result.numel() < 3 or not result.is_contiguous():
+        raise ValueError("result must be a contiguous int32 tensor of at least 3 elements")
+    if result.device != dev:
+        raise ValueError("result must be on the current device")
+    _check(load().tp_diag_bounded_wait(int(limit_us), result.data_ptr(), _stream(stream)),
+           "tp_diag_bounded_wait")
 
 
 def tp_set_decode_max_tokens(max_tokens: int) -> None:

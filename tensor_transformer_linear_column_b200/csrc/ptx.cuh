@@ -67,15 +67,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase of `bar` with parity `parity` has completed.
 // Returns false (after flagging the error and raising *abort) if the wait runs
-// past the limit, or at once if *abort is already raised by another role.
-__device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, volatile int* abort) {
+// past `limit_ns`, or at once if *abort is already raised by another role.
+__device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, volatile int* abort,
+                                            unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(&g_tp_device_error, kErrTimeout);
         return false;
@@ -349,6 +350,10 @@ __device__ __forceinline__ void cluster_sync_all() {
 // memory (local and remote) writes before the arrival with reads after the wait.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void cluster_wait_acquire() {

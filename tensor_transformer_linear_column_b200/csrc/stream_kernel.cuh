@@ -34,10 +34,14 @@
 // (st.async, cluster scope) whose bytes complete on an mbarrier in the owner;
 // each owner waits for exactly those bytes, sums the csize partials of its rows
 // in a fixed order from its own shared memory, adds the bias, applies the
-// activation and stores bf16.  A CTA keeps no buffer alive for its peers, so it
-// exits as soon as its own rows are stored.  Nothing intermediate goes to
-// global memory and there are no atomics, so the result is bit-identical from
-// run to run for a given shape and t.
+// activation and stores bf16.  A split cluster barrier closes the exchange:
+// every thread arrives once it has issued its last remote store, and a CTA
+// waits for that phase before it reads its receive buffer and before it exits,
+// so no CTA leaves while a peer may still write into its shared memory, also
+// when a bounded wait has run out somewhere in the cluster (every wait before a
+// send is bounded, so the phase always completes).  Nothing intermediate goes
+// to global memory and there are no atomics, so the result is bit-identical
+// from run to run for a given shape and t.
 //
 // Weight traffic: a ring of 2-8 stages of one or two k-blocks each (3-D TMA
 // boxes), deeper for CTAs that stream longer.  With static weights the first
@@ -553,18 +557,24 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     tc_fence_before();
   }
   if (multi && warp == kStreamProducerWarp) cluster_wait_acquire();  // phase 1 (sends nothing)
+  // cluster phase 2: "this thread has issued its last remote store".  Warps 0-3
+  // arrive after their sends; the others have none.
+  if (multi) cluster_arrive_release();
 
   __syncthreads();
   if (warp == kStreamMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_d, tcols_alloc);
   }
-  if (!multi || warp >= 4) return;
+  if (!multi) return;
+  // no CTA of the cluster exits, and no owner reads its receive buffer, before
+  // every peer has issued all of its remote stores
+  cluster_wait_acquire();
+  if (warp >= 4) return;
 
   // ---------------- owner: fixed-order sum of the csize partials of its rows.
-  // Every peer always sends its T values per row, so this completes within
-  // microseconds; once it has, nothing in the cluster touches this CTA's shared
-  // memory again and the CTA may exit without a closing cluster barrier.
+  // Every peer always sends its T values per row and has issued them by now,
+  // so this completes within microseconds.
   if (!drain_wait(smem_u32(recv_bar), 0, 50ull * 1000ull * 1000ull))
     atomicOr(&g_tp_device_error, kErrTimeout);
   const int RS = stream_recv_stride(p.T);

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "diag_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "ptx.cuh"
 #include "stream_kernel.cuh"
@@ -692,6 +693,15 @@ tp_status tp_device_error_check(void) {
     return TP_ERR_DEVICE_TIMEOUT;
   }
   return TP_OK;
+}
+
+tp_status tp_diag_bounded_wait(unsigned int limit_us, int* result, tp_stream_t stream) {
+  if (result == nullptr) return TP_ERR_NULL;
+  if (!aligned16(result)) return TP_ERR_ALIGN;
+  if (limit_us < 1u || limit_us > 1000000u) return TP_ERR_UNSUPPORTED;
+  tpb::bounded_wait_probe_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull, result);
+  return cuda_ok(cudaGetLastError(), "launch bounded_wait_probe_kernel") ? TP_OK : TP_ERR_CUDA;
 }
 
 tp_status tp_set_decode_max_tokens(int max_tokens) {

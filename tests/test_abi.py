@@ -229,28 +229,16 @@ def test_launch_options_setting(lib):
 
 # ---------------------------------------------------------------- launch plans (host only)
 
-def _profile_row(path, metric):
-    """The three per-launch values of `metric` in a committed ncu summary table."""
-    with open(path) as f:
-        for line in f:
-            if line.startswith(f"| `{metric}` |"):
-                cells = [c.strip() for c in line.strip().strip("|").split("|")[1:]]
-                return [float(c.split()[0]) for c in cells]
-    raise AssertionError(f"{metric} not in {path}")
-
-
-def test_stream_plan_matches_the_profiled_sq4096_launches():
-    # the committed ncu capture of the 4096 x 4096 decode step (T = 1, 8, 64)
-    # records what the GPU launched; the host plan must still produce it
-    path = os.path.join(ROOT, "profiles", "stream_gemm_kernel_sq4096.md")
-    smem_kb = _profile_row(path, "launch__shared_mem_per_block_dynamic")
-    grid = _profile_row(path, "launch__grid_size")
-    cluster = _profile_row(path, "launch__cluster_dim_y")
-    for i, T in enumerate((1, 8, 64)):
+def test_stream_plan_of_the_sq4096_decode_launches():
+    # the launches the GPU made for the 4096 x 4096 decode step (T = 1, 8, 64),
+    # as an ncu capture recorded them: 32 n-tiles x clusters of 8 CTAs along K,
+    # dynamic shared memory per CTA in bytes
+    expected = {1: (256, 8, 58512), 8: (256, 8, 60560), 64: (256, 8, 109712)}
+    for T, (grid, cluster, smem) in expected.items():
         p = tp.tp_stream_plan(T, 4096, 4096)
-        assert p["smem_bytes"] == round(smem_kb[i] * 1000)
-        assert p["grid_x"] * p["cluster"] == grid[i]
-        assert p["cluster"] == cluster[i]
+        assert p["grid_x"] * p["cluster"] == grid
+        assert p["cluster"] == cluster
+        assert p["smem_bytes"] == smem
 
 
 def test_stream_plan_ring_depths_of_the_70b_decode():

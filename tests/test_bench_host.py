@@ -80,3 +80,22 @@ def test_reference_arm_times_the_oracle_on_cpu(capsys):
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["metric"] == bench.METRIC
+
+
+def test_default_workload_is_the_405b_block():
+    # the N = 1 line is the whole block on the largest single-GPU workload
+    args = bench.parse([])
+    assert args.workload == "mlp405b"
+    assert args.steps >= 1 and args.warmup >= 3
+    # about a second of timed work at ~25 ms per step
+    assert 20 <= args.steps <= 200
+    args = bench.parse(["--workload", "sq4096"])
+    assert args.steps >= 1000
+
+
+def test_reference_and_device_arms_share_the_config():
+    # the reference line names the same workload, split, L2 policy and options
+    c = bench.workload_config("mlp405b", 8, "pdl+static_weights")
+    assert c["name"] == "mlp405b" and c["tp_degree"] == 8 and c["tokens"] == [8192]
+    assert "read once per step" in c["l2"] and c["launch_options"] == "pdl+static_weights"
+    assert bench.rotation_copies(bench.workload_weight_bytes("sq4096")) == 16

@@ -259,6 +259,39 @@ def test_attn70b_prefill_sampled_rows():
     assert torch.isfinite(y.float()).all() and torch.isfinite(qkv.float()).all()
 
 
+@pytest.fixture(scope="module")
+def attn70b_weights():
+    cfg = workloads.CONFIGS["attn70b"]
+    d = workloads.attn_inputs(cfg, 1, with_bias=True)
+    return cfg, d
+
+
+@pytest.mark.parametrize("T", [1, 16, 64])
+@pytest.mark.parametrize("bias", [False, True])
+def test_attn70b_decode_projections(attn70b_weights, T, bias):
+    # decode-shaped calls of the attention projections on the 70B head layout
+    # (64 query / 8 key-value heads of 128, t = 8): both go through the
+    # weight-streaming kernel -- QKV N = 10240 column-parallel, O-projection
+    # over nctx = 8192 with 8 head-group shards of 1024
+    dev = _dev()
+    cfg, d = attn70b_weights
+    nq, nkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    x = workloads.random_bf16_small((T, cfg.hidden), 1.0, 300 + T)
+    ctx = workloads.random_bf16_small((T, nq * hd), 1.0, 400 + T)
+    b_qkv = d["b_qkv"] if bias else None
+    b_o = d["b_o"] if bias else None
+    q_ref = oracle.attn_qkv(x, d["w_qkv"], b_qkv, nq, nkv, hd, 8)
+    o_ref = oracle.attn_out(ctx, d["w_o"], b_o, nq, hd, 8)
+    with launch_options(BENCH_OPTIONS):
+        qkv, y = tp.tp_attn_proj_forward(x.to(dev), d["w_qkv"].to(dev), _cuda(b_qkv, dev),
+                                         ctx.to(dev), d["w_o"].to(dev), _cuda(b_o, dev),
+                                         nq, nkv, hd, 8)
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert_parity(qkv, q_ref, f"attn70b decode qkv T={T}")
+    assert_parity(y, o_ref, f"attn70b decode out T={T}")
+
+
 def test_mlp405b_prefill_sampled_rows():
     dev = _dev()
     cfg = workloads.CONFIGS["mlp405b"]

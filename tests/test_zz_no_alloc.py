@@ -4,16 +4,20 @@ belongs to another allocator, loops that cannot take cudaMalloc's implicit
 synchronisation).
 
 tp_mlp_forward_noalloc keeps the activation between the two layers in the
-library's own static device array instead of a caller workspace.  These tests
-call it through the C ABI and check it against tp_mlp_forward (the workspace
-entry point) with the parity tolerance used everywhere else, on two calls in a
-row, on both kernel paths, and check that sizes past the array are refused.
-This file is collected last on purpose.
+library's own static device array instead of a caller workspace.  It runs the
+same kernels with the same launch geometry as tp_mlp_forward (the workspace
+entry point), so these tests call both through the C ABI and require the two
+results to be bit-identical, on two calls in a row, on both kernel paths (a
+stale or misaligned read of the array would shift a few ulps, which a
+tolerance would hide); each result is also held to the parity tolerance used
+everywhere else against the fp64 oracle.  Sizes past the array must be
+refused.  This file is collected last on purpose.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import tensor_transformer_linear_column_b200 as tp
 import workloads
 
@@ -49,7 +53,11 @@ def test_noalloc_matches_workspace_call_twice(T, H, F, t):
         ref = tp.tp_mlp_forward(x, w1, b1, w2, b2, t, "gelu_tanh")
         y = tp.tp_mlp_forward_noalloc(x, w1, b1, w2, b2, t, "gelu_tanh")
         torch.cuda.synchronize()
-        _close(y, ref, f"call {call} T={T} F={F}")
+        assert torch.equal(y, ref), f"call {call} T={T} F={F}: not bit-identical"
+        if call == 0:
+            exact = oracle.mlp_block(x.cpu(), w1.cpu(), b1.cpu(), w2.cpu(), b2.cpu(), t,
+                                     "gelu_tanh")
+            _close(y, torch.from_numpy(exact), f"call {call} T={T} F={F} vs oracle")
     assert tp.tp_device_error_check() == tp.TP_OK
 
 
