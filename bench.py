@@ -631,8 +631,8 @@ def roofline(wl, ms_per_step, stream, use_graph, power_capped=False):
 
 
 def kernel_durations(wl, stream, reps=5):
-    """Average duration of each kernel of a prefill step, timed alone with events
-    (T > 128: both GEMMs run on the CTA-pair kernel)."""
+    """Average duration of each kernel of a prefill step, each launch between its
+    own events (T > 128: both GEMMs run on the CTA-pair kernel)."""
     tp = wl.tp
     T = wl.Ts[0]
     out = {}
@@ -660,17 +660,23 @@ def kernel_durations(wl, stream, reps=5):
                 lambda: tp.tp_rowpar_gemm_reduce(h, w2, wl.bias[1], wl.t, out=wl.outs[T]),
                 2 * T * F * H),
         }
-    for name, (fn, flops) in calls.items():
-        with torch.cuda.stream(stream):
-            fn()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                fn()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        out[name] = (e0.elapsed_time(e1) / reps, flops)
+    # the kernels of the step are timed interleaved (a, b, a, b, ...), each
+    # between its own events, so both see the same clocks and power state
+    names = list(calls)
+    with torch.cuda.stream(stream):
+        for name in names:
+            calls[name][0]()
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)] for _ in names]
+        for r in range(reps):
+            for i, name in enumerate(names):
+                ev[i][r][0].record(stream)
+                calls[name][0]()
+                ev[i][r][1].record(stream)
+    torch.cuda.synchronize()
+    for i, name in enumerate(names):
+        ms = sum(a.elapsed_time(b) for a, b in ev[i]) / reps
+        out[name] = (ms, calls[name][1])
     return out
 
 
