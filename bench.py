@@ -196,7 +196,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs of one workload and its step as C-ABI calls."""
 
-    def __init__(self, name: str, tp_degree, device, rotate=True):
+    def __init__(self, name: str, tp_degree, device, rotate=True, tokens=None):
         import tensor_transformer_linear_column_b200 as tp
         self.tp = tp
         self.name = name
@@ -205,7 +205,7 @@ class Workload:
         cfg = self.cfg
         if name == "sq4096":
             self.t = tp_degree or cfg.tp_degrees[0]
-            self.Ts = list(cfg.tokens)
+            self.Ts = list(tokens or cfg.tokens)
             w = workloads.proj_inputs(cfg, 1)["w"]
             self.weight_bytes = w.numel() * 2
             self.xs = {T: workloads.normal_bf16((T, cfg.k), 1.0, 0, workloads.x_index(T))
@@ -215,7 +215,7 @@ class Workload:
             self.bias = None
         elif name in ("tiny", "mlp70b", "mlp405b"):
             self.t = tp_degree or cfg.tp_degrees[-1]
-            self.Ts = list(cfg.tokens)
+            self.Ts = list(tokens or cfg.tokens)
             d = workloads.mlp_inputs(cfg, self.Ts[0])
             self.xs = {T: workloads.mlp_x(cfg, T) for T in self.Ts}
             self.weight_bytes = (d["w1"].numel() + d["w2"].numel()) * 2
@@ -227,7 +227,7 @@ class Workload:
                                   dtype=torch.uint8, device=device)
         elif name == "mlp70b_w8":
             self.t = tp_degree or cfg.tp_degrees[-1]
-            self.Ts = list(cfg.tokens)
+            self.Ts = list(tokens or cfg.tokens)
             d = workloads.mlp_inputs(cfg, self.Ts[0])
             self.xs = {T: workloads.mlp_x(cfg, T) for T in self.Ts}
             q1, s1 = workloads.quantize_e4m3_rows(d["w1"])
@@ -240,7 +240,7 @@ class Workload:
                                   dtype=torch.uint8, device=device)
         elif name == "attn70b":
             self.t = tp_degree or cfg.tp_degrees[0]
-            self.Ts = list(cfg.tokens)
+            self.Ts = list(tokens or cfg.tokens)
             d = workloads.attn_inputs(cfg, self.Ts[0])
             self.xs = {self.Ts[0]: d["x"]}
             self.ctx = d["ctx"].to(device)
@@ -471,7 +471,7 @@ def rotation_copies(weight_bytes):
     return 1
 
 
-def workload_config(name, t, options):
+def workload_config(name, t, options, tokens=None):
     cfg = workloads.CONFIGS[name]
     desc = {
         "sq4096": "column-parallel projection W[4096,4096] bf16, t=2 column shards, decode T=1,8,64",
@@ -486,7 +486,9 @@ def workload_config(name, t, options):
     }[name]
     wb = workload_weight_bytes(name)
     rot = rotation_copies(wb)
-    return {"workload": desc, "name": name, "tp_degree": t, "tokens": list(cfg.tokens),
+    if tokens:
+        desc += f" (token counts overridden: {list(tokens)})"
+    return {"workload": desc, "name": name, "tp_degree": t, "tokens": list(tokens or cfg.tokens),
             "parallelism": "replicas (per-GPU block, t logical shards on chip)",
             "l2": (f"weights rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
                    f"the 126 MB L2): every call reads cold weights" if rot > 1 else
@@ -503,7 +505,7 @@ def run_ours(args, world, rank, local):
     init_dist(world, "nccl")
     tp.load()
     tp.tp_set_launch_options(LAUNCH_OPTIONS[args.options])
-    wl = Workload(args.workload, args.tp, dev, rotate=True)
+    wl = Workload(args.workload, args.tp, dev, rotate=True, tokens=args.tokens)
     stream = torch.cuda.Stream(device=dev)
     K, W = args.steps, args.warmup
 
@@ -576,7 +578,7 @@ def run_ours(args, world, rank, local):
     e2e = end_to_end(wl, stream, max(3, min(K, args.e2e_steps)), world, dev)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.tokens:
         v, steps, el, toks = time_oracle(args.workload, args.tp, budget_s=args.cpu_budget)
         cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{steps} full oracle step(s) of {toks} tokens in {el:.1f} s "
@@ -588,7 +590,7 @@ def run_ours(args, world, rank, local):
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0, sigma) bf16 inputs of the workload's shapes)",
-            "config": workload_config(args.workload, wl.t, args.options),
+            "config": workload_config(args.workload, wl.t, args.options, args.tokens),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": wl.launches_per_step * K,
             "clocks": clocks,
@@ -727,6 +729,9 @@ def parse(argv=None):
     ap.add_argument("--options", choices=sorted(LAUNCH_OPTIONS), default="pdl+static_weights",
                     help="library launch options: the workload's weights are loaded once and "
                          "never written, so kernels may prefetch them under PDL")
+    ap.add_argument("--tokens", type=int, nargs="+", default=None,
+                    help="override the workload's token counts (smaller captures for ncu); "
+                         "not a headline configuration")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -170,6 +170,43 @@ tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_
                                tp_stream_t stream);
 
 /*
+ * Bytes of workspace tp_mlp_backward needs: three [T, F] bf16 activations (the
+ * pre-activation z, its gradient dz and h = act(z)), each rounded up to 256
+ * bytes.  Returns 0 for T < 1 or F < 1.
+ */
+size_t tp_mlp_backward_workspace_bytes(int T, int F);
+
+/*
+ * Backward pass of the tensor-parallel MLP block (tp_mlp_forward) for an
+ * upstream gradient dy = dL/dy.  The split needs two more all-reduces per layer
+ * in the backward pass (xingyuzhitong.com "Tensor vs Pipeline Parallelism",
+ * section "Tensor parallelism: split inside each layer"); for the MLP the one
+ * that carries data is the sum over shards of the input gradient, since every
+ * column shard used all of x.  dy reaches every shard whole, and each weight
+ * gradient stays on the shard that owns the weight:
+ *   z    = x w1^T + b1                      (recomputed, column-parallel)
+ *   dz   = (dy w2) * act'(z),  h = act(z)    shard s: columns F_s, no exchange
+ *   dx   = ((dz[:,F_0] w1[F_0,:] + dz[:,F_1] w1[F_1,:]) + ...)   fused shard sum,
+ *          each partial from zero, ascending shard order
+ *   dw1  = dz^T x [F, H],   dw2 = dy^T h [H, F]   (contractions over tokens)
+ *   db1  = sum over tokens of dz [F],  db2 = sum over tokens of dy [H]
+ * Arithmetic: bf16 operands, fp32 accumulation; z, dz and h are rounded to
+ * bf16 once, in the workspace; every output is rounded once to bf16.
+ *   x [T, H], w1 [F, H], b1 [F] or NULL, w2 [H, F], dy [T, H]    (read)
+ *   dx [T, H], dw1 [F, H], dw2 [H, F]                           (written)
+ *   db1 [F], db2 [H]: written unless NULL
+ *   workspace: at least tp_mlp_backward_workspace_bytes(T, F) bytes, 16-byte
+ *   aligned; on return it holds z, dz and h (in that order, each in its
+ *   256-byte-rounded slot).
+ * Requires F % t == 0 and (F / t) % 64 == 0; T >= 1 is arbitrary.
+ */
+tp_status tp_mlp_backward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                          const tp_bf16* w2, const tp_bf16* dy,
+                          int T, int H, int F, int tp_degree, int act,
+                          tp_bf16* dx, tp_bf16* dw1, tp_bf16* db1, tp_bf16* dw2, tp_bf16* db2,
+                          void* workspace, size_t workspace_bytes, tp_stream_t stream);
+
+/*
  * Largest activation h[T, F] (T * F * 2 bytes) that tp_mlp_forward_noalloc can
  * hold: 4 MiB, e.g. 64 tokens at F = 28672 or 2048 tokens at F = 1024.
  */

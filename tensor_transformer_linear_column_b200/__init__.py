@@ -45,6 +45,9 @@ SIGNATURES = {
     "tp_mlp_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "tp_mlp_backward_workspace_bytes": (_Z, [_I, _I]),
+    "tp_mlp_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
+                             _P]),
     "tp_colpar_gemm_gelu_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "tp_rowpar_gemm_reduce_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "tp_mlp_forward_w8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
@@ -233,6 +236,41 @@ def tp_mlp_forward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor]
                                int(tp_degree), _act(act), _ptr(out, "out", dev),
                                workspace.data_ptr(), ws_bytes, _stream(stream))
     _check(st, "tp_mlp_forward")
+    return out
+
+
+def tp_mlp_backward_workspace_bytes(T: int, F: int) -> int:
+    return int(load().tp_mlp_backward_workspace_bytes(int(T), int(F)))
+
+
+def tp_mlp_backward(x: torch.Tensor, w1: torch.Tensor, b1: Optional[torch.Tensor],
+                    w2: torch.Tensor, dy: torch.Tensor, tp_degree: int, act="gelu_tanh",
+                    with_bias_grads: bool = True, workspace: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of the tensor-parallel MLP block for the upstream gradient dy:
+    {"dx", "dw1", "db1", "dw2", "db2"} (the bias gradients only if asked)."""
+    T, H = x.shape
+    F = w1.shape[0]
+    if w1.shape[1] != H or tuple(w2.shape) != (H, F) or tuple(dy.shape) != (T, H):
+        raise ValueError("w1 must be [F, H], w2 [H, F] and dy [T, H]")
+    dev = _device(x)
+    out = {"dx": torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+           "dw1": torch.empty((F, H), dtype=torch.bfloat16, device=dev),
+           "dw2": torch.empty((H, F), dtype=torch.bfloat16, device=dev),
+           "db1": torch.empty((F,), dtype=torch.bfloat16, device=dev) if with_bias_grads else None,
+           "db2": torch.empty((H,), dtype=torch.bfloat16, device=dev) if with_bias_grads else None}
+    need = tp_mlp_backward_workspace_bytes(T, F)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the same device")
+    st = load().tp_mlp_backward(
+        _ptr(x, "x", dev), _ptr(w1, "w1", dev), _ptr(b1, "b1", dev), _ptr(w2, "w2", dev),
+        _ptr(dy, "dy", dev), T, H, F, int(tp_degree), _act(act), _ptr(out["dx"], "dx", dev),
+        _ptr(out["dw1"], "dw1", dev), _ptr(out["db1"], "db1", dev), _ptr(out["dw2"], "dw2", dev),
+        _ptr(out["db2"], "db2", dev), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "tp_mlp_backward")
     return out
 
 

@@ -22,6 +22,15 @@
 // (xingyuzhitong.com "Tensor vs Pipeline Parallelism", section "Tensor
 // parallelism: split inside each layer": the partial results of the
 // row-split layer are summed).
+//
+// Operand layouts (template flags kAmn, kBmn): an operand is K-major (the
+// forward pass: activations [rows, K] and weights [out, in]) or MN-major, read
+// straight from a row-major [K][MN] matrix with no transpose in memory (the
+// backward pass: dy W2 reads W2 [H, F] with F as N; dz^T x reads dz [T, F] and
+// x [T, H] with the tokens as K).  An MN-major 128-row operand half arrives as
+// two TMA boxes of 64 MN x 64 K.  The backward pass's third epilogue
+// (kEpiDact) multiplies the product by act'(z) for a stored pre-activation z
+// and also writes act(z).
 #pragma once
 
 #include "ptx.cuh"
@@ -39,12 +48,77 @@ constexpr int kPairStageBytes = 2 * kPairHalfBytes;       // own A rows + own B 
 constexpr int kPairTmemCols = 2 * kPairBN;                // two 256-column accumulators
 constexpr int kPairSmemBytes = 1024 + kPairStages * kPairStageBytes + (2 * kPairStages + 5) * 8 + 16;
 
+// epilogues: bias + activation (one segment per tile), the row-parallel shard
+// sum (t segments per tile), and the activation gradient (one segment)
+constexpr int kEpiAct = 0;
+constexpr int kEpiRowpar = 1;
+constexpr int kEpiDact = 2;
+
+// 32 fp32 products g at columns [col, col + 32) of one row, and the stored
+// pre-activations z at the same places: dst = g * act'(z), dst2 = act(z)
+// (act = none: dst = g, dst2 = z), each rounded once to bf16.
+__device__ __forceinline__ void store_row_chunk32_dact(uint16_t* dst, uint16_t* dst2,
+                                                       const uint16_t* z_chunk,
+                                                       const float (&g)[32], int act) {
+  const uint4* zp = reinterpret_cast<const uint4*>(z_chunk);
+  uint32_t pd[16], ph[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(zp + q);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int j = q * 8 + h * 2;
+      const float z0 = __uint_as_float(w4[h] << 16);
+      const float z1 = __uint_as_float(w4[h] & 0xFFFF0000u);
+      float a0 = z0, a1 = z1, d0 = 1.0f, d1 = 1.0f;
+      if (act == 1) {
+        gelu_tanh_and_grad_f32(z0, a0, d0);
+        gelu_tanh_and_grad_f32(z1, a1, d1);
+      }
+      pd[q * 4 + h] = pack_bf16x2(g[j] * d0, g[j + 1] * d1);
+      ph[q * 4 + h] = pack_bf16x2(a0, a1);
+    }
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  uint4* h4 = reinterpret_cast<uint4*>(dst2);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    d4[q] = make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+    h4[q] = make_uint4(ph[4 * q], ph[4 * q + 1], ph[4 * q + 2], ph[4 * q + 3]);
+  }
+}
+
+// Load this CTA's 128 rows of one operand for k-block kb into `dst` (16 KB):
+// K-major, one box {64 K, 128 rows} at (kb * 64, row0); MN-major, two boxes
+// {64 MN, 64 K} at (row0, kb * 64) and (row0 + 64, kb * 64), 8 KB apart.
+template <bool kMn>
+__device__ __forceinline__ void pair_load_half(uint32_t dst, const CUtensorMap* map,
+                                               uint32_t bar_cluster, int kb, int row0) {
+  if constexpr (kMn) {
+    tma_load_2d_pair(dst, map, bar_cluster, row0, kb * kPairBK);
+    tma_load_2d_pair(dst + kPairHalfBytes / 2, map, bar_cluster, row0 + 64, kb * kPairBK);
+  } else {
+    tma_load_2d_pair(dst, map, bar_cluster, kb * kPairBK, row0);
+  }
+}
+
+// Descriptor of MMA step kk (K = 16) of a 128-row operand half at `base`.
+template <bool kMn>
+__device__ __forceinline__ uint64_t pair_desc(uint32_t base, int kk) {
+  if constexpr (kMn)
+    return desc_mnmajor_sw128(base + static_cast<uint32_t>(kk) * 2048u, kPairHalfBytes / 2);
+  else
+    return desc_kmajor_sw128(base + static_cast<uint32_t>(kk) * 32u);
+}
+
 // 320 threads: registers are granted per group of four warps, so the ten warps
 // count as twelve and 168 registers per thread is the ceiling.
-template <bool kRowpar>
+template <int kEpi, bool kAmn, bool kBmn>
 __global__ void __launch_bounds__(kPairThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b, const TiledParams p) {
+  constexpr bool kRowpar = kEpi == kEpiRowpar;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -112,8 +186,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kb = 0; kb < pre; ++kb) {
           const uint32_t sa = smem_u32(smem + kb * kPairStageBytes);
           if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[kb]), 2 * kPairStageBytes);
-          tma_load_2d_pair(sa + kPairHalfBytes, &tmap_b, leader_full0 + kb * 8, kb * kPairBK,
-                           n0 * kPairBN + half_row);
+          pair_load_half<kBmn>(sa + kPairHalfBytes, &tmap_b, leader_full0 + kb * 8, kb,
+                               n0 * kPairBN + half_row);
           issued |= 1u << kb;
         }
       }
@@ -126,7 +200,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint32_t ph = static_cast<uint32_t>(it / kPairStages) & 1u;
           const uint32_t sa = smem_u32(smem + s * kPairStageBytes);
           if (it < pre) {  // weight half already requested
-            tma_load_2d_pair(sa, &tmap_a, leader_full0 + s * 8, kb * kPairBK, m * kPairBM + half_row);
+            pair_load_half<kAmn>(sa, &tmap_a, leader_full0 + s * 8, kb, m * kPairBM + half_row);
             continue;
           }
           if (!wait_parity(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag)) {
@@ -134,9 +208,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             break;
           }
           if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * kPairStageBytes);
-          tma_load_2d_pair(sa, &tmap_a, leader_full0 + s * 8, kb * kPairBK, m * kPairBM + half_row);
-          tma_load_2d_pair(sa + kPairHalfBytes, &tmap_b, leader_full0 + s * 8, kb * kPairBK,
-                           n * kPairBN + half_row);
+          pair_load_half<kAmn>(sa, &tmap_a, leader_full0 + s * 8, kb, m * kPairBM + half_row);
+          pair_load_half<kBmn>(sa + kPairHalfBytes, &tmap_b, leader_full0 + s * 8, kb,
+                               n * kPairBN + half_row);
           issued |= 1u << s;
           phases = (phases & ~(1u << s)) | (ph << s);
         }
@@ -159,7 +233,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer for the pair (leader only)
-      const uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN);
+      const uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN, kAmn, kBmn);
       int it = 0, acc = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < p.tiles; tile += npairs) {
@@ -183,9 +257,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint32_t sa = smem_u32(smem + s * kPairStageBytes);
 #pragma unroll
             for (int kk = 0; kk < kPairBK / 16; ++kk) {
-              umma_bf16_pair(d, desc_kmajor_sw128(sa + kk * 32),
-                             desc_kmajor_sw128(sa + kPairHalfBytes + kk * 32), idesc,
-                             (kb > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16_pair(d, pair_desc<kAmn>(sa, kk), pair_desc<kBmn>(sa + kPairHalfBytes, kk),
+                             idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit_pair(smem_u32(&empty_bar[s]), 0x3);
           }
@@ -241,9 +314,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
             const int col = col0 + c * 32;
-            if (row < p.M && col < p.N)
-              store_row_chunk32(p.out + static_cast<size_t>(row) * p.N + col, v,
-                                p.bias != nullptr ? p.bias + col : nullptr, p.act);
+            if (row < p.M && col < p.N) {
+              const size_t off = static_cast<size_t>(row) * p.N + col;
+              if constexpr (kEpi == kEpiDact)
+                store_row_chunk32_dact(p.out + off, p.out2 + off, p.aux + off, v, p.act);
+              else
+                store_row_chunk32(p.out + off, v, p.bias != nullptr ? p.bias + col : nullptr,
+                                  p.act);
+            }
           }
         } else {
 #pragma unroll

@@ -162,11 +162,30 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D.
+// Descriptor for an MN-major bf16 operand written by TMA with 128-byte
+// swizzling from a row-major [K][MN] global matrix in boxes of 64 MN x 64 K:
+// each K index is a 128-byte row of 64 consecutive MN elements, 8 such rows
+// form a 1024-byte core group (stride offset 1024 between K groups), and the
+// next 64 MN elements are `lbo` bytes further (leading offset).  One MMA step
+// of K = 16 spans two core groups, so step kk starts 2048 kk bytes in.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D.
 // D format [4,6)=1 (f32), A format [7,10)=1 (bf16), B format [10,13)=1,
-// N>>3 at [17,23), M>>4 at [24,29).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+// A major [15] and B major [16] (0 = K-major, 1 = MN-major), N>>3 at
+// [17,23), M>>4 at [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false,
+                                                      bool b_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -424,6 +443,20 @@ __device__ __forceinline__ float gelu_tanh_f32(float z) {
   const float k1 = 0.044715f;
   const float u = k0 * fmaf(k1 * z, z * z, z);
   return 0.5f * z * (1.0f + tanh_approx(u));
+}
+
+// The tanh-form GeLU and its derivative at z, from one tanh: with
+// u = c (z + a z^3) and th = tanh u, g = 0.5 z (1 + th) and
+// g' = 0.5 (1 + th) + 0.5 z (1 - th^2) c (1 + 3 a z^2)
+// (product and chain rules applied to the form above).
+__device__ __forceinline__ void gelu_tanh_and_grad_f32(float z, float& g, float& dg) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
+  const float k1 = 0.044715f;
+  const float z2 = z * z;
+  const float th = tanh_approx(k0 * fmaf(k1 * z, z2, z));
+  const float half1 = 0.5f * (1.0f + th);
+  g = z * half1;
+  dg = fmaf(0.5f * z * (1.0f - th * th), k0 * fmaf(3.0f * k1, z2, 1.0f), half1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -53,6 +53,9 @@ struct TiledParams {
   int prefetch_w;  // issue the first stages' weight (B) loads before waiting for the previous grid
   const uint16_t* bias;  // [N] or nullptr
   uint16_t* out;         // [M, N]
+  // activation-gradient epilogue of the CTA-pair kernel only:
+  const uint16_t* aux;   // [M, N] pre-activation z the gradient flows through
+  uint16_t* out2;        // [M, N] act(z), written beside the gradient
 };
 
 __device__ __forceinline__ void tiled_coords(int tile, const TiledParams& p, int& m, int& n) {

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "colsum_kernel.cuh"
 #include "diag_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "ptx.cuh"
@@ -79,6 +80,25 @@ bool stream_attrs(StreamKernel k, int smem) {
                  "cudaFuncSetAttribute");
 }
 
+// The CTA-pair kernel's instantiations: (epilogue, A MN-major, B MN-major).
+using PairKernel = void (*)(const CUtensorMap, const CUtensorMap, const tpb::TiledParams);
+constexpr PairKernel kPairKernels[] = {
+    tpb::pair_gemm_kernel<tpb::kEpiAct, false, false>,     // forward column-parallel
+    tpb::pair_gemm_kernel<tpb::kEpiRowpar, false, false>,  // forward row-parallel + sum
+    tpb::pair_gemm_kernel<tpb::kEpiDact, false, true>,     // dy W2, times act'(z)
+    tpb::pair_gemm_kernel<tpb::kEpiRowpar, false, true>,   // sum_s dz_s W1_s
+    tpb::pair_gemm_kernel<tpb::kEpiAct, true, true>,       // weight gradients (K = tokens)
+};
+
+PairKernel pair_kernel_for(int epi, bool a_mn, bool b_mn) {
+  if (!a_mn && !b_mn) return epi == tpb::kEpiAct ? kPairKernels[0]
+                             : epi == tpb::kEpiRowpar ? kPairKernels[1] : nullptr;
+  if (!a_mn && b_mn) return epi == tpb::kEpiDact ? kPairKernels[2]
+                            : epi == tpb::kEpiRowpar ? kPairKernels[3] : nullptr;
+  if (a_mn && b_mn && epi == tpb::kEpiAct) return kPairKernels[4];
+  return nullptr;
+}
+
 const DeviceInfo* device_info() {
   int dev = 0;
   if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -107,15 +127,11 @@ const DeviceInfo* device_info() {
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            tpb::kTiledSmemBytes), "cudaFuncSetAttribute"))
     return nullptr;
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::pair_gemm_kernel<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    tpb::kPairSmemBytes),
-               "cudaFuncSetAttribute") ||
-      !cuda_ok(cudaFuncSetAttribute(tpb::pair_gemm_kernel<true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    tpb::kPairSmemBytes),
-               "cudaFuncSetAttribute"))
-    return nullptr;
+  for (PairKernel k : kPairKernels)
+    if (!cuda_ok(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      tpb::kPairSmemBytes),
+                 "cudaFuncSetAttribute"))
+      return nullptr;
   d.sms = sms;
   d.max_smem = smem;
   d.ready = true;
@@ -349,30 +365,47 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   return TP_OK;
 }
 
-// Persistent CTA-pair kernel (256 x 256 tiles on two SMs).
-tp_status launch_pair(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
-                      const tp_bf16* b, int M, int K, int N, int segs, int act, tp_bf16* out,
-                      cudaStream_t stream) {
+// One operand of the CTA-pair kernel as it is stored: K-major ([rows, K],
+// K contiguous) or MN-major ([K, rows], the rows' index contiguous).
+struct PairOperand {
+  const tp_bf16* ptr;
+  bool mn;
+};
+
+// Persistent CTA-pair kernel (256 x 256 tiles on two SMs): out[M, N] =
+// epilogue(A[M, K] B[N, K]^T).  K need not be a multiple of 64: the loads
+// past K read zeros.  `prefetch` allows B's first k-blocks to be requested
+// before the preceding grid completes (B is a weight that no kernel writes).
+tp_status launch_pair_ex(const DeviceInfo& dev, PairOperand a, PairOperand bop, const tp_bf16* bias,
+                         int M, int K, int N, int segs, int epi, int act, tp_bf16* out,
+                         const tp_bf16* aux, tp_bf16* out2, bool prefetch, cudaStream_t stream) {
+  const PairKernel kernel = pair_kernel_for(epi, a.mn, bop.mn);
+  if (kernel == nullptr) return TP_ERR_UNSUPPORTED;
   TiledParams p{};
   p.M = M;
   p.N = N;
   p.K = K;
-  p.kb_total = K / tpb::kPairBK;
+  p.kb_total = (K + tpb::kPairBK - 1) / tpb::kPairBK;
   p.segs = segs;
   p.m_tiles = (M + tpb::kPairBM - 1) / tpb::kPairBM;
   p.n_tiles = (N + tpb::kPairBN - 1) / tpb::kPairBN;
   p.tiles = p.m_tiles * p.n_tiles;
   p.group_m = p.m_tiles < 8 ? p.m_tiles : 8;
   p.act = act;
-  p.prefetch_w = prefetch_weights();
-  p.bias = b;
+  p.prefetch_w = prefetch ? prefetch_weights() : 0;
+  p.bias = bias;
   p.out = out;
+  p.aux = aux;
+  p.out2 = out2;
 
+  // K-major: box {64 K, 128 rows} of [rows, K]; MN-major: box {64 rows, 64 K} of [K, rows]
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, a, static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128))
-    return TP_ERR_CUDA;
-  if (!make_tmap(&tb, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K), 128))
-    return TP_ERR_CUDA;
+  const bool ta_ok = a.mn ? make_tmap(&ta, a.ptr, static_cast<uint64_t>(K), static_cast<uint64_t>(M), 64)
+                          : make_tmap(&ta, a.ptr, static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128);
+  if (!ta_ok) return TP_ERR_CUDA;
+  const bool tb_ok = bop.mn ? make_tmap(&tb, bop.ptr, static_cast<uint64_t>(K), static_cast<uint64_t>(N), 64)
+                            : make_tmap(&tb, bop.ptr, static_cast<uint64_t>(N), static_cast<uint64_t>(K), 128);
+  if (!tb_ok) return TP_ERR_CUDA;
 
   const int pairs = p.tiles < dev.sms / 2 ? p.tiles : dev.sms / 2;
   cudaLaunchConfig_t cfg{};
@@ -387,12 +420,17 @@ tp_status launch_pair(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 1));
-  cudaError_t e;
-  if (segs > 1)
-    e = cudaLaunchKernelEx(&cfg, tpb::pair_gemm_kernel<true>, ta, tb, p);
-  else
-    e = cudaLaunchKernelEx(&cfg, tpb::pair_gemm_kernel<false>, ta, tb, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, p);
   return cuda_ok(e, "launch pair_gemm_kernel") ? TP_OK : TP_ERR_CUDA;
+}
+
+// The forward pass's use of it: K-major activations and weights.
+tp_status launch_pair(const DeviceInfo& dev, const tp_bf16* a, const tp_bf16* w,
+                      const tp_bf16* b, int M, int K, int N, int segs, int act, tp_bf16* out,
+                      cudaStream_t stream) {
+  return launch_pair_ex(dev, PairOperand{a, false}, PairOperand{w, false}, b, M, K, N, segs,
+                        segs > 1 ? tpb::kEpiRowpar : tpb::kEpiAct, act, out, nullptr, nullptr,
+                        true, stream);
 }
 
 // Persistent tiled kernel.  segs = t accumulation segments in row-parallel
@@ -575,6 +613,68 @@ tp_status tp_attn_proj_forward(const tp_bf16* x, const tp_bf16* w_qkv, const tp_
   tp_status s = run_colpar(x, w_qkv, b_qkv, T, H, static_cast<int>(nqkv), TP_ACT_NONE, qkv_out, st);
   if (s != TP_OK) return s;
   return run_rowpar(ctx, w_o, b_o, T, static_cast<int>(nctx), H, tp_degree, out, st);
+}
+
+size_t tp_mlp_backward_workspace_bytes(int T, int F) {
+  if (T < 1 || F < 1) return 0;
+  return 3u * tp_mlp_workspace_bytes(T, F);
+}
+
+tp_status tp_mlp_backward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                          const tp_bf16* w2, const tp_bf16* dy, int T, int H, int F,
+                          int tp_degree, int act, tp_bf16* dx, tp_bf16* dw1, tp_bf16* db1,
+                          tp_bf16* dw2, tp_bf16* db2, void* workspace, size_t workspace_bytes,
+                          tp_stream_t stream) {
+  if (x == nullptr || w1 == nullptr || w2 == nullptr || dy == nullptr || dx == nullptr ||
+      dw1 == nullptr || dw2 == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(dy) || !aligned16(dx) ||
+      !aligned16(dw1) || !aligned16(dw2) || (b1 != nullptr && !aligned16(b1)) ||
+      (db1 != nullptr && !aligned16(db1)) || (db2 != nullptr && !aligned16(db2)))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || !feat_ok(F)) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_TANH) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || F % tp_degree != 0 || (F / tp_degree) % 64 != 0) return TP_ERR_TP_DEGREE;
+  if (workspace == nullptr || workspace_bytes < tp_mlp_backward_workspace_bytes(T, F))
+    return TP_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TP_ERR_ALIGN;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t slot = tp_mlp_workspace_bytes(T, F);
+  tp_bf16* z = static_cast<tp_bf16*>(workspace);
+  tp_bf16* dz = reinterpret_cast<tp_bf16*>(static_cast<uint8_t*>(workspace) + slot);
+  tp_bf16* h = reinterpret_cast<tp_bf16*>(static_cast<uint8_t*>(workspace) + 2 * slot);
+  // z = x W1^T + b1, the forward pre-activation (column-parallel, no activation)
+  tp_status s = run_colpar(x, w1, b1, T, H, F, TP_ACT_NONE, z, st);
+  if (s != TP_OK) return s;
+  // dz = (dy W2) * act'(z) and h = act(z); W2 [H, F] is read with F as N (MN-major).
+  // Shard s's columns F_s need nothing from other shards: dy reaches every shard whole.
+  s = launch_pair_ex(*dev, PairOperand{dy, false}, PairOperand{w2, true}, nullptr, T, H, F, 1,
+                     tpb::kEpiDact, act, dz, z, h, true, st);
+  if (s != TP_OK) return s;
+  // dx = sum_s dz[:, F_s] W1[F_s, :]: the backward all-reduce, each shard's
+  // partial from zero, summed in ascending shard order in the epilogue
+  s = launch_pair_ex(*dev, PairOperand{dz, false}, PairOperand{w1, true}, nullptr, T, F, H,
+                     tp_degree, tpb::kEpiRowpar, TP_ACT_NONE, dx, nullptr, nullptr, true, st);
+  if (s != TP_OK) return s;
+  // weight gradients stay on their shards: dW1 = dz^T x [F, H], dW2 = dy^T h [H, F],
+  // contractions over the tokens (both operands read MN-major)
+  s = launch_pair_ex(*dev, PairOperand{dz, true}, PairOperand{x, true}, nullptr, F, T, H, 1,
+                     tpb::kEpiAct, TP_ACT_NONE, dw1, nullptr, nullptr, false, st);
+  if (s != TP_OK) return s;
+  s = launch_pair_ex(*dev, PairOperand{dy, true}, PairOperand{h, true}, nullptr, H, T, F, 1,
+                     tpb::kEpiAct, TP_ACT_NONE, dw2, nullptr, nullptr, false, st);
+  if (s != TP_OK) return s;
+  if (db1 != nullptr) {
+    tpb::colsum_kernel<<<(F + 63) / 64, tpb::kColsumWarps * 32, 0, st>>>(dz, T, F, db1);
+    if (!cuda_ok(cudaGetLastError(), "launch colsum_kernel")) return TP_ERR_CUDA;
+  }
+  if (db2 != nullptr) {
+    tpb::colsum_kernel<<<(H + 63) / 64, tpb::kColsumWarps * 32, 0, st>>>(dy, T, H, db2);
+    if (!cuda_ok(cudaGetLastError(), "launch colsum_kernel")) return TP_ERR_CUDA;
+  }
+  return TP_OK;
 }
 
 tp_status tp_colpar_gemm_gelu_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,

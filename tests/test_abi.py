@@ -157,6 +157,29 @@ def test_mlp_rejects_bad_arguments(lib):
     assert call(F=1000) == tp.TP_ERR_SHAPE
 
 
+def test_backward_rejects_bad_arguments(lib):
+    def call(x=GOOD, dy=GOOD, dx=GOOD, dw1=GOOD, dw2=GOOD, db1=None, ws=GOOD,
+             ws_bytes=1 << 22, T=8, H=256, F=1024, t=2, act=1):
+        return lib.tp_mlp_backward(x, GOOD, None, GOOD, dy, T, H, F, t, act, dx, dw1, db1, dw2,
+                                   None, ws, ws_bytes, None)
+    assert tp.tp_mlp_backward_workspace_bytes(8, 1024) == 3 * 8 * 1024 * 2
+    assert tp.tp_mlp_backward_workspace_bytes(3, 64) == 3 * 512
+    assert tp.tp_mlp_backward_workspace_bytes(0, 64) == 0
+    assert call(x=None) == tp.TP_ERR_NULL
+    assert call(dy=None) == tp.TP_ERR_NULL
+    assert call(dw2=None) == tp.TP_ERR_NULL
+    assert call(dx=ODD) == tp.TP_ERR_ALIGN
+    assert call(db1=ODD) == tp.TP_ERR_ALIGN
+    assert call(T=0) == tp.TP_ERR_SHAPE
+    assert call(H=100) == tp.TP_ERR_SHAPE
+    assert call(act=4) == tp.TP_ERR_UNSUPPORTED
+    assert call(t=3) == tp.TP_ERR_TP_DEGREE
+    assert call(t=32) == tp.TP_ERR_TP_DEGREE
+    assert call(ws=None) == tp.TP_ERR_WORKSPACE
+    assert call(ws_bytes=3 * 8 * 1024 * 2 - 1) == tp.TP_ERR_WORKSPACE
+    assert call(ws=ODD) == tp.TP_ERR_ALIGN
+
+
 def test_attention_head_rules_from_the_pages(lib, golden):
     g = golden["head_divisibility"]
 
