@@ -207,6 +207,51 @@ tp_status tp_mlp_backward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1
                           void* workspace, size_t workspace_bytes, tp_stream_t stream);
 
 /*
+ * Bytes of workspace tp_attn_decode needs for T new tokens after `past` cached
+ * ones (the per-chunk partial results); 0 for unsupported arguments.  A
+ * function of the sizes only.
+ */
+size_t tp_attn_decode_workspace_bytes(int T, int past, int n_q_heads, int n_kv_heads,
+                                      int head_dim);
+
+/*
+ * The attention core between the two projections of tp_attn_proj_forward, for
+ * decode: T new tokens of one sequence attend over its key-value cache.
+ * Attention heads are distributed among the tensor-parallel shards, each with
+ * its share of the KV cache, so the core needs no exchange (xingyuzhitong.com
+ * "Tensor vs Pipeline Parallelism", section "Tensor parallelism: split inside
+ * each layer"; drpranayjha.com "AI Infrastructure series, Part 5", section "How
+ * does tensor parallelism split a layer?"): shard s owns query heads
+ * [s nq/t, (s+1) nq/t), key-value heads [s nkv/t, (s+1) nkv/t) and their cache
+ * rows.  On one GPU the shards are head groups of one grid.
+ *   1. the new tokens' keys and values (columns K and V of qkv) are written
+ *      into the cache at positions [past, past + T);
+ *   2. ctx[i, h d .. h d + d) = sum_j p_j v_j over keys j <= past + i of
+ *      key-value head g = h / (nq / nkv), with p = softmax_j(q_i,h . k_j / sqrt(d))
+ *      (causal, grouped-query; no positional rotation is applied here).
+ * Arithmetic: bf16 q, k, v; scores, maxima and sums in fp32; the softmax
+ * weights are rounded to bf16 for the weighted sum of v (fp32 accumulate) and
+ * their row sum is taken from the rounded weights; the keys are processed in
+ * chunks whose partial results are merged in a fixed chunk order, so the
+ * result is bit-identical from run to run and does not depend on the GPU.
+ *   qkv      [T, (nq + 2 nkv) d]  tp_attn_proj_forward's qkv_out   (read)
+ *   k_cache  [nkv, max_len, d]    rows [0, past) hold the cached keys;
+ *                                 rows [past, past + T) are written
+ *   v_cache  [nkv, max_len, d]    likewise for values
+ *   ctx      [T, nq d]            the input of the output projection (written)
+ *   workspace: at least tp_attn_decode_workspace_bytes(...) bytes, 16-byte
+ *   aligned; contents on return unspecified.
+ * Requires head_dim == 128 (else TP_ERR_UNSUPPORTED), nq / nkv in {1, 2, 4,
+ * 8, 16} (else TP_ERR_UNSUPPORTED), past + T <= max_len (else TP_ERR_SHAPE),
+ * and t dividing both head counts (else TP_ERR_TP_DEGREE).  Calls that
+ * overlap on the GPU must not share a workspace or a cache.
+ */
+tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache, int T, int past,
+                         int max_len, int n_q_heads, int n_kv_heads, int head_dim, int tp_degree,
+                         tp_bf16* ctx, void* workspace, size_t workspace_bytes,
+                         tp_stream_t stream);
+
+/*
  * Largest activation h[T, F] (T * F * 2 bytes) that tp_mlp_forward_noalloc can
  * hold: 4 MiB, e.g. 64 tokens at F = 28672 or 2048 tokens at F = 1024.
  */

@@ -46,6 +46,8 @@ SIGNATURES = {
     "tp_attn_proj_forward": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "tp_mlp_backward_workspace_bytes": (_Z, [_I, _I]),
+    "tp_attn_decode_workspace_bytes": (_Z, [_I, _I, _I, _I, _I]),
+    "tp_attn_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_mlp_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
                              _P]),
     "tp_colpar_gemm_gelu_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
@@ -395,6 +397,42 @@ def tp_attn_proj_forward(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: Optional[t
                                      _ptr(out, "out", dev), _stream(stream))
     _check(st, "tp_attn_proj_forward")
     return qkv_out, out
+
+
+def tp_attn_decode_workspace_bytes(T: int, past: int, n_q_heads: int, n_kv_heads: int,
+                                   head_dim: int) -> int:
+    return int(load().tp_attn_decode_workspace_bytes(int(T), int(past), int(n_q_heads),
+                                                     int(n_kv_heads), int(head_dim)))
+
+
+def tp_attn_decode(qkv: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, past: int,
+                   n_q_heads: int, n_kv_heads: int, head_dim: int, tp_degree: int,
+                   ctx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """ctx [T, nq d] of T new tokens (qkv [T, (nq + 2 nkv) d]) over the caches
+    k_cache, v_cache [nkv, max_len, d] holding `past` tokens; appends the new
+    tokens' keys and values to the caches in place."""
+    T = qkv.shape[0]
+    if qkv.shape[1] != (n_q_heads + 2 * n_kv_heads) * head_dim:
+        raise ValueError("qkv must be [T, (nq + 2 nkv) d]")
+    if k_cache.dim() != 3 or tuple(k_cache.shape) != tuple(v_cache.shape) or \
+            k_cache.shape[0] != n_kv_heads or k_cache.shape[2] != head_dim:
+        raise ValueError("caches must be [nkv, max_len, d]")
+    dev = _device(qkv)
+    if ctx is None:
+        ctx = torch.empty((T, n_q_heads * head_dim), dtype=torch.bfloat16, device=dev)
+    need = tp_attn_decode_workspace_bytes(T, past, n_q_heads, n_kv_heads, head_dim)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    if workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the same device")
+    st = load().tp_attn_decode(_ptr(qkv, "qkv", dev), _ptr(k_cache, "k_cache", dev),
+                               _ptr(v_cache, "v_cache", dev), T, int(past), k_cache.shape[1],
+                               int(n_q_heads), int(n_kv_heads), int(head_dim), int(tp_degree),
+                               _ptr(ctx, "ctx", dev), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "tp_attn_decode")
+    return ctx
 
 
 def tp_device_error_check() -> int:

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "attn_kernel.cuh"
 #include "colsum_kernel.cuh"
 #include "diag_kernel.cuh"
 #include "pair_kernel.cuh"
@@ -132,6 +133,10 @@ const DeviceInfo* device_info() {
                                       tpb::kPairSmemBytes),
                  "cudaFuncSetAttribute"))
       return nullptr;
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_decode_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+               "cudaFuncSetAttribute"))
+    return nullptr;
   d.sms = sms;
   d.max_smem = smem;
   d.ready = true;
@@ -531,6 +536,76 @@ tp_status run_linear_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scal
   return launch_stream(*dev, g, x, w8, w_scale, b, T, K, N, shards, act, out, stream);
 }
 
+// ------------------------------------------------------------------ attention core (decode)
+
+// The launch of the decode attention core for a shape; a function of the shape
+// only (not of the device), so the chunking and therefore the order of the
+// sums are the same on every GPU.  TP_ERR_UNSUPPORTED if G is not 1, 2, 4, 8
+// or 16.
+constexpr int kAttnTargetCtas = 296;  // two waves' worth of CTAs on 148 SMs
+
+tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& groups,
+                    size_t& part_o_bytes, size_t& part_ml_bytes) {
+  const int G = nq / nkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return TP_ERR_UNSUPPORTED;
+  p = tpb::AttnParams{};
+  p.T = T;
+  p.past = past;
+  p.L = past + T;
+  p.nq = nq;
+  p.nkv = nkv;
+  p.G = G;
+  // At most 32 query rows per CTA: the scores of a whole chunk (up to 8 key
+  // blocks) then fit in TMEM, so the chunk maximum is known before any P V
+  // product and no accumulator is rescaled.  More tokens form token groups
+  // (grid z), each of which reads the chunk's keys and values again.
+  const int tq_step = G >= 16 ? 1 : 16 / G;   // tokens that make 16 query rows
+  const int tq_max = 32 / G;
+  if (T <= tq_max) {
+    p.Tq = (T + tq_step - 1) / tq_step * tq_step;
+    groups = 1;
+  } else {
+    p.Tq = tq_max;
+    groups = (T + tq_max - 1) / tq_max;
+  }
+  p.n_pad = p.Tq * G;
+  const int nblk = (p.L + tpb::kAttnBlockKeys - 1) / tpb::kAttnBlockKeys;
+  // S of every block of a chunk plus O in at most 256 TMEM columns
+  int nb_max = 256 / p.n_pad - 1;
+  nb_max = nb_max < 1 ? 1 : (nb_max > 8 ? 8 : nb_max);
+  int nb = (nkv * groups * nblk + kAttnTargetCtas - 1) / kAttnTargetCtas;
+  nb = nb < 1 ? 1 : (nb > nb_max ? nb_max : nb);
+  p.nb = nb;
+  p.chunks = (nblk + nb - 1) / nb;
+  p.tmem_cols = next_pow2((nb + 1) * p.n_pad < 32 ? 32 : (nb + 1) * p.n_pad);
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(tpb::kAttnHeadDim));
+  const size_t rows = static_cast<size_t>(groups) * nkv * p.chunks * p.n_pad;
+  part_o_bytes = (rows * tpb::kAttnHeadDim * 4 + 255) / 256 * 256;
+  part_ml_bytes = (rows * 2 * 4 + 255) / 256 * 256;
+  return TP_OK;
+}
+
+// 3-D view {d, rows, outer} of a bf16 tensor whose rows are d = 128 elements
+// apart and whose outer index is `outer_stride` elements apart; a box
+// {64, box_rows, box_outer} lands as box_outer * box_rows 128-byte rows with
+// 128-byte swizzling.  Reads outside [0, rows) return zeros.
+bool make_tmap_rows3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t outer,
+                     uint64_t row_stride, uint64_t outer_stride, uint32_t box_rows,
+                     uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_ok(cudaErrorSymbolNotFound, "cuTensorMapEncodeTiled lookup");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(tpb::kAttnHeadDim), rows, outer};
+  cuuint64_t strides[2] = {row_stride * 2, outer_stride * 2};
+  cuuint32_t box[3] = {64, box_rows, box_outer};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (rows3)");
+  return ok;
+}
+
 // ------------------------------------------------------------------ checks
 
 tp_status check_linear(const void* x, const void* w, const void* b, const void* out, int T, int K,
@@ -673,6 +748,111 @@ tp_status tp_mlp_backward(const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1
   if (db2 != nullptr) {
     tpb::colsum_kernel<<<(H + 63) / 64, tpb::kColsumWarps * 32, 0, st>>>(dy, T, H, db2);
     if (!cuda_ok(cudaGetLastError(), "launch colsum_kernel")) return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
+size_t tp_attn_decode_workspace_bytes(int T, int past, int n_q_heads, int n_kv_heads,
+                                      int head_dim) {
+  if (T < 1 || past < 0 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads != 0 ||
+      head_dim != tpb::kAttnHeadDim)
+    return 0;
+  tpb::AttnParams p;
+  int groups = 0;
+  size_t po = 0, pml = 0;
+  if (plan_attn(T, past, n_q_heads, n_kv_heads, p, groups, po, pml) != TP_OK) return 0;
+  return po + pml;
+}
+
+tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache, int T, int past,
+                         int max_len, int n_q_heads, int n_kv_heads, int head_dim, int tp_degree,
+                         tp_bf16* ctx, void* workspace, size_t workspace_bytes,
+                         tp_stream_t stream) {
+  if (qkv == nullptr || k_cache == nullptr || v_cache == nullptr || ctx == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(ctx))
+    return TP_ERR_ALIGN;
+  if (T < 1 || past < 0 || n_q_heads < 1 || n_kv_heads < 1 || head_dim < 1 ||
+      n_q_heads % n_kv_heads != 0 || max_len < 1 || static_cast<long long>(past) + T > max_len ||
+      static_cast<long long>(n_kv_heads) * max_len * head_dim > (1ll << 40))
+    return TP_ERR_SHAPE;
+  if (head_dim != tpb::kAttnHeadDim) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || n_q_heads % tp_degree != 0 || n_kv_heads % tp_degree != 0)
+    return TP_ERR_TP_DEGREE;
+  tpb::AttnParams p;
+  int groups = 0;
+  size_t po = 0, pml = 0;
+  const tp_status planned = plan_attn(T, past, n_q_heads, n_kv_heads, p, groups, po, pml);
+  if (planned != TP_OK) return planned;
+  if (workspace == nullptr || workspace_bytes < po + pml) return TP_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TP_ERR_ALIGN;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  const int smem = tpb::attn_smem_bytes(p.nb, p.n_pad);
+  if (smem > dev->max_smem) return TP_ERR_UNSUPPORTED;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + po);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int nqkv = (n_q_heads + 2 * n_kv_heads) * head_dim;
+
+  // Q: {d, heads, tokens}; K, V: {d, keys 0 .. L - 1, key-value heads}
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_rows3(&tq, qkv, static_cast<uint64_t>(n_q_heads), static_cast<uint64_t>(T),
+                       static_cast<uint64_t>(head_dim), static_cast<uint64_t>(nqkv),
+                       static_cast<uint32_t>(p.G), static_cast<uint32_t>(p.Tq)) ||
+      !make_tmap_rows3(&tk, k_cache, static_cast<uint64_t>(p.L), static_cast<uint64_t>(n_kv_heads),
+                       static_cast<uint64_t>(head_dim),
+                       static_cast<uint64_t>(max_len) * head_dim, tpb::kAttnBlockKeys, 1) ||
+      !make_tmap_rows3(&tv, v_cache, static_cast<uint64_t>(p.L), static_cast<uint64_t>(n_kv_heads),
+                       static_cast<uint64_t>(head_dim),
+                       static_cast<uint64_t>(max_len) * head_dim, tpb::kAttnBlockKeys, 1))
+    return TP_ERR_CUDA;
+
+  cudaLaunchAttribute attr[1];
+  const int nattr = launch_attrs(attr, 0);
+  // 1. the new tokens' keys and values into the cache
+  {
+    const int total = T * n_kv_heads * (tpb::kAttnHeadDim / 8) * 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>((total + 255) / 256), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(nattr);
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::kv_append_kernel, qkv, k_cache, v_cache, T, past,
+                                    max_len, n_q_heads, n_kv_heads),
+                 "launch kv_append_kernel"))
+      return TP_ERR_CUDA;
+  }
+  // 2. chunk partials: grid (chunks, key-value heads, token groups)
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.chunks), static_cast<unsigned>(n_kv_heads),
+                       static_cast<unsigned>(groups));
+    cfg.blockDim = dim3(tpb::kAttnThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(nattr);
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel, tq, tk, tv, p),
+                 "launch attn_decode_kernel"))
+      return TP_ERR_CUDA;
+  }
+  // 3. merge the chunks of every (token, query head) in chunk order
+  {
+    const int warps = T * n_q_heads;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + 7) / 8), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(nattr);
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::attn_combine_kernel,
+                                    static_cast<const float*>(p.part_o),
+                                    static_cast<const float*>(p.part_ml), T, n_q_heads,
+                                    n_kv_heads, p.G, p.Tq, p.n_pad, p.chunks, ctx),
+                 "launch attn_combine_kernel"))
+      return TP_ERR_CUDA;
   }
   return TP_OK;
 }

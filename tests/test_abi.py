@@ -180,6 +180,28 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(ws=ODD) == tp.TP_ERR_ALIGN
 
 
+def test_attn_decode_rejects_bad_arguments(lib):
+    def call(qkv=GOOD, kc=GOOD, ctx=GOOD, T=1, past=10, max_len=64, nq=64, nkv=8, d=128, t=8,
+             ws=GOOD, ws_bytes=1 << 24):
+        return lib.tp_attn_decode(qkv, kc, GOOD, T, past, max_len, nq, nkv, d, t, ctx, ws,
+                                  ws_bytes, None)
+    assert tp.tp_attn_decode_workspace_bytes(1, 10, 64, 8, 128) > 0
+    assert tp.tp_attn_decode_workspace_bytes(1, 10, 64, 8, 64) == 0      # d must be 128
+    assert tp.tp_attn_decode_workspace_bytes(1, 10, 24, 8, 128) == 0     # G = 3
+    assert call(qkv=None) == tp.TP_ERR_NULL
+    assert call(kc=ODD) == tp.TP_ERR_ALIGN
+    assert call(T=0) == tp.TP_ERR_SHAPE
+    assert call(past=60, T=5) == tp.TP_ERR_SHAPE                       # past + T > max_len
+    assert call(nq=60) == tp.TP_ERR_SHAPE                              # nkv does not divide nq
+    assert call(d=64) == tp.TP_ERR_UNSUPPORTED
+    assert call(nq=24) == tp.TP_ERR_UNSUPPORTED                        # G = 3
+    assert call(t=3) == tp.TP_ERR_TP_DEGREE
+    assert call(t=16) == tp.TP_ERR_TP_DEGREE                           # 8 kv heads: t <= 8
+    assert call(ws=None) == tp.TP_ERR_WORKSPACE
+    assert call(ws_bytes=tp.tp_attn_decode_workspace_bytes(1, 10, 64, 8, 128) - 1) == \
+        tp.TP_ERR_WORKSPACE
+
+
 def test_attention_head_rules_from_the_pages(lib, golden):
     g = golden["head_divisibility"]
 
