@@ -54,11 +54,13 @@ KERNEL_SOURCES = {
     "stream_gemm_kernel": ["csrc/ptx.cuh", "csrc/stream_kernel.cuh"],
     "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh"],
     "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh"],
+    "attn_decode_kernel": ["csrc/ptx.cuh", "csrc/attn_kernel.cuh"],
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # default (timed steps, warm-up steps) per workload: about a second of timed work
-DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "mlp70b": (2000, 50),
+DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "attn70b_decode": (5000, 50),
+                 "mlp70b": (2000, 50),
                  "mlp70b_w8": (2000, 50), "sq4096": (20000, 200), "tiny": (20000, 200)}
 
 
@@ -249,6 +251,24 @@ class Workload:
             self.weights = [(d["w_qkv"].to(device), d["w_o"].to(device))]
             nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
             self.qkv = torch.empty((self.Ts[0], nqkv), dtype=torch.bfloat16, device=device)
+        elif name == "attn70b_decode":
+            self.t = tp_degree or cfg.tp_degrees[0]
+            self.Ts = list(tokens or cfg.tokens)
+            self.xs = {T: workloads.attn_decode_qkv(cfg, T) for T in self.Ts}
+            k, v = workloads.attn_decode_cache(cfg)
+            d = cfg.head_dim
+            self.max_len = cfg.past + max(self.Ts)
+            kc = torch.empty((cfg.n_kv_heads, self.max_len, d), dtype=torch.bfloat16, device=device)
+            vc = torch.empty_like(kc)
+            kc[:, :cfg.past].copy_(k)
+            vc[:, :cfg.past].copy_(v)
+            self.weights = [(kc, vc)]
+            self.weight_bytes = 2 * k.numel() * 2  # the cache read by every call
+            self.hidden_in = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * d
+            self.hidden_out = cfg.n_q_heads * d
+            self.ws = torch.empty(max(tp.tp_attn_decode_workspace_bytes(
+                T, cfg.past, cfg.n_q_heads, cfg.n_kv_heads, d) for T in self.Ts),
+                dtype=torch.uint8, device=device)
         else:
             raise ValueError(name)
         self.xd = {T: x.to(device) for T, x in self.xs.items()}
@@ -265,7 +285,7 @@ class Workload:
                 else:
                     self.weights.append(base.clone())
         self.tokens_per_step = sum(self.Ts)
-        self.launches_per_step = len(self.Ts) * (1 if name == "sq4096" else 2)
+        self.launches_per_step = len(self.Ts) * {"sq4096": 1, "attn70b_decode": 3}.get(name, 2)
 
     def step(self, i: int, xs=None, outs=None):
         tp = self.tp
@@ -280,6 +300,10 @@ class Workload:
             elif self.name == "mlp70b_w8":
                 tp.tp_mlp_forward_w8(xs[T], w[0], w[1], None, w[2], w[3], None, self.t,
                                      self.cfg.act, out=outs[T], workspace=self.ws)
+            elif self.name == "attn70b_decode":
+                c = self.cfg
+                tp.tp_attn_decode(xs[T], w[0], w[1], c.past, c.n_q_heads, c.n_kv_heads,
+                                  c.head_dim, self.t, ctx=outs[T], workspace=self.ws)
             elif self.name == "attn70b":
                 tp.tp_attn_proj_forward(xs[T], w[0], None, self.ctx, w[1], None,
                                         self.cfg.n_q_heads, self.cfg.n_kv_heads,
@@ -294,6 +318,9 @@ class Workload:
         b = 0
         for T in self.Ts:
             b += self.weight_bytes + 2 * T * (self.hidden_in + self.hidden_out)
+            if self.name == "attn70b_decode":
+                # the new tokens' keys and values: written to the cache, then read
+                b += 2 * 2 * 2 * T * self.cfg.n_kv_heads * self.cfg.head_dim
             if self.name in ("tiny", "mlp70b", "mlp70b_w8", "mlp405b"):
                 b += 2 * 2 * T * self.cfg.ffn  # h written and read once
         return b
@@ -307,6 +334,9 @@ class Workload:
 
     def bound(self):
         return "tensor" if max(self.Ts) > 256 else "hbm"
+
+    def hbm_kernel(self):
+        return "attn_decode_kernel" if self.name == "attn70b_decode" else "stream_gemm_kernel"
 
 
 class _OracleRunner:
@@ -323,7 +353,12 @@ class _OracleRunner:
         cfg = workloads.CONFIGS[name]
         self.name = name
         self.cfg = cfg
-        if name == "sq4096":
+        if name == "attn70b_decode":
+            self.t = t or cfg.tp_degrees[0]
+            self.xs = {T: workloads.attn_decode_qkv(cfg, T) for T in cfg.tokens}
+            self.k, self.v = workloads.attn_decode_cache(cfg)
+            self.n_out = cfg.n_q_heads * cfg.head_dim
+        elif name == "sq4096":
             self.t = t or cfg.tp_degrees[0]
             self.w = workloads.proj_inputs(cfg, 1)["w"]
             self.xs = {T: workloads.normal_bf16((T, cfg.k), 1.0, 0, workloads.x_index(T))
@@ -362,6 +397,15 @@ class _OracleRunner:
     def run(self, fraction, offset):
         """Compute the step on output-feature block [offset, offset + fraction * n_out)."""
         import oracle
+        if self.name == "attn70b_decode":
+            # every new token needs the whole cache: the sample is whole calls
+            c = self.cfg
+            kh = c.n_kv_heads // self.t
+            cache = [(self.k[s * kh:(s + 1) * kh], self.v[s * kh:(s + 1) * kh])
+                     for s in range(self.t)]
+            for T, qkv in self.xs.items():
+                oracle.attn_core(qkv, c.n_q_heads, c.n_kv_heads, c.head_dim, self.t, cache)
+            return 1.0
         n = self.n_out
         cnt = max(64, int(round(fraction * n)) // 64 * 64)
         j0 = (offset * cnt) % n
@@ -461,6 +505,8 @@ def workload_weight_bytes(name):
         return (nqkv + cfg.n_q_heads * cfg.head_dim) * cfg.hidden * 2
     if name == "mlp70b_w8":
         return 2 * cfg.hidden * cfg.ffn + 4 * (cfg.hidden + cfg.ffn)
+    if name == "attn70b_decode":
+        return 2 * cfg.n_kv_heads * cfg.past * cfg.head_dim * 2
     return 2 * cfg.hidden * cfg.ffn * 2
 
 
@@ -481,18 +527,21 @@ def workload_config(name, t, options, tokens=None):
                      "8-bit weights (FP8 E4M3 codes, one fp32 scale per row)",
         "attn70b": "Llama-3-70B-shaped attention projections prefill T=4096, QKV 8192->10240 "
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
+        "attn70b_decode": "attention core decode, 64 query / 8 key-value heads of 128 (t=8), "
+                          "65536 cached tokens, T=1,2,4 new tokens per call",
         "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192, column-parallel "
                    "up-projection + row-parallel down-projection with the fused 8-shard sum",
     }[name]
     wb = workload_weight_bytes(name)
     rot = rotation_copies(wb)
+    what = "KV caches" if name == "attn70b_decode" else "weights"
     if tokens:
         desc += f" (token counts overridden: {list(tokens)})"
     return {"workload": desc, "name": name, "tp_degree": t, "tokens": list(tokens or cfg.tokens),
             "parallelism": "replicas (per-GPU block, t logical shards on chip)",
-            "l2": (f"weights rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
-                   f"the 126 MB L2): every call reads cold weights" if rot > 1 else
-                   f"weights {wb / 1e6:.0f} MB > 126 MB L2, read once per step"),
+            "l2": (f"{what} rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
+                   f"the 126 MB L2): every call reads cold {what}" if rot > 1 else
+                   f"{what} {wb / 1e6:.0f} MB > 126 MB L2, read once per step"),
             "launch_options": options}
 
 
@@ -612,10 +661,11 @@ def roofline(wl, ms_per_step, stream, use_graph, power_capped=False):
         peak = float(peaks["hbm_gbs"])
         unit = "GB/s"
         launches = wl.launches_per_step
-        traffic = recorded_traffic("stream_gemm_kernel", wl.name)
+        kernel = wl.hbm_kernel()
+        traffic = recorded_traffic(kernel, wl.name)
         return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "stream_gemm_kernel", "launches_per_step": launches,
+                "kernel": kernel, "launches_per_step": launches,
                 "bytes_per_step": wl.step_bytes(), "peak_source": f"{src} hbm_gbs"}
     # tensor-bound: time each kernel of the step alone with events on the stream
     per_kernel = kernel_durations(wl, stream)

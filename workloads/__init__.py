@@ -132,6 +132,18 @@ class AttnConfig:
     sample_rows: Optional[int] = None
 
 
+@dataclasses.dataclass(frozen=True)
+class AttnDecodeConfig:
+    """The attention core in decode: new tokens over a per-head KV cache."""
+    name: str
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    past: int               # cached tokens before the new ones
+    tokens: Tuple[int, ...]  # new tokens per call, one call per entry
+    tp_degrees: Tuple[int, ...]
+
+
 CONFIGS: Dict[str, object] = {
     # x[8,256] fp32, W1[256->1024], W2[1024->256] N(0,0.02), biases N(0,0.01), t=2
     "tiny": MLPConfig("tiny", hidden=256, ffn=1024, tokens=(8,), tp_degrees=(2,),
@@ -150,6 +162,10 @@ CONFIGS: Dict[str, object] = {
     "attn70b": AttnConfig("attn70b", hidden=8192, n_q_heads=64, n_kv_heads=8,
                           head_dim=128, tokens=(4096,), tp_degrees=(8,), w_std=0.02,
                           sample_rows=64),
+    # the attention core between the 70B projections, decode over a 64K-token cache
+    "attn70b_decode": AttnDecodeConfig("attn70b_decode", n_q_heads=64, n_kv_heads=8,
+                                       head_dim=128, past=65536, tokens=(1, 2, 4),
+                                       tp_degrees=(8,)),
     # 405B-shaped MLP prefill; the oracle checks 64 seeded rows
     "mlp405b": MLPConfig("mlp405b", hidden=16384, ffn=53248, tokens=(8192,),
                          tp_degrees=(8,), act="gelu_tanh", w_std=0.01, b_std=None,
@@ -210,6 +226,20 @@ def attn_inputs(cfg: AttnConfig, T: int, seed: int = 0, with_bias: bool = False
     b_qkv = normal_bf16((nqkv,), 0.01, seed, IDX_QKV_B) if with_bias else None
     b_o = normal_bf16((H,), 0.01, seed, IDX_O_B) if with_bias else None
     return {"x": x, "w_qkv": w_qkv, "b_qkv": b_qkv, "ctx": ctx, "w_o": w_o, "b_o": b_o}
+
+
+def attn_decode_qkv(cfg: AttnDecodeConfig, T: int, seed: int = 0) -> torch.Tensor:
+    """qkv [T, (nq + 2 nkv) d] of T new tokens, N(0, 1) bf16 (the projections'
+    outputs have no fixed scale; unit variance keeps the scores q.k / sqrt(d)
+    of order one)."""
+    nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    return normal_bf16((T, nqkv), 1.0, seed, 500 + int(T))
+
+
+def attn_decode_cache(cfg: AttnDecodeConfig, seed: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The caches k, v [nkv, past, d] of the cached tokens, N(0, 1) bf16."""
+    shape = (cfg.n_kv_heads, cfg.past, cfg.head_dim)
+    return normal_bf16(shape, 1.0, seed, 601), normal_bf16(shape, 1.0, seed, 602)
 
 
 def quantize_e4m3_rows(w: torch.Tensor, rows_per_chunk: int = 2048
