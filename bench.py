@@ -622,6 +622,8 @@ def run_ours(args, world, rank, local):
     # kernel attribution: each kernel type of the step timed alone (same inputs)
     power_capped = bool(clocks and "sw_power_cap" in clocks.get("reasons", []))
     roof = roofline(wl, ms_per_step, stream, use_graph, power_capped)
+    if args.tokens:
+        roof["traffic"] = None  # recorded captures are per launch of the workload's own sizes
 
     # end to end through the public API with host buffers (pinned)
     e2e = end_to_end(wl, stream, max(3, min(K, args.e2e_steps)), world, dev)
