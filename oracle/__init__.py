@@ -24,3 +24,11 @@ from .tp_oracle import (  # noqa: F401
 )
 from .tp_attention import attend_head, attn_core, empty_cache  # noqa: F401
 from .tp_backward import act_grad, gelu_tanh_grad, mlp_block_backward  # noqa: F401
+from .tp_sequence import (  # noqa: F401
+    RMS_EPS,
+    all_gather,
+    reduce_scatter,
+    rms_norm,
+    sp_residual_norm,
+    token_shards,
+)
