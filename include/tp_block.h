@@ -252,6 +252,33 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                          tp_stream_t stream);
 
 /*
+ * The sequence-parallel region after a row-parallel linear: residual add and
+ * RMSNorm, token shard by token shard.  Sequence parallelism splits the parts
+ * of a layer that tensor parallelism leaves whole (normalisation, dropout)
+ * along the sequence inside the tensor-parallel group (drpranayjha.com "AI
+ * Infrastructure series, Part 5", section "What about MoE models and very long
+ * prompts?"): the row-parallel all-reduce becomes a reduce-scatter that leaves
+ * shard s the summed rows of its tokens [s T/t, (s+1) T/t), the shard adds
+ * the residual stream and normalises its rows, and an all-gather returns every
+ * token for the next column-parallel linear.  On one GPU tp_rowpar_gemm_reduce
+ * has already summed every row (the reduce-scatter and the all-gather together
+ * are that all-reduce), so this call is the per-shard region itself:
+ *   r_out = residual + y
+ *   n_out = r / sqrt(mean_j r_j^2 + eps) * gamma      (RMSNorm of each token row)
+ * Arithmetic: fp32 from the bf16 inputs; n is computed from the fp32 r; each
+ * output is rounded once to bf16; the sum of squares is taken in a fixed order.
+ *   y [T, H] (the row-parallel output), residual [T, H], gamma [H]  (read)
+ *   r_out [T, H], n_out [T, H]                                       (written)
+ *   eps >= 0 (1e-5 for Llama-shaped models)
+ * Requires T % t == 0 (equal token shards; else TP_ERR_TP_DEGREE) and H a
+ * positive multiple of 64.  Dropout is the identity at inference and is not
+ * applied.
+ */
+tp_status tp_sp_add_rmsnorm(const tp_bf16* y, const tp_bf16* residual, const tp_bf16* gamma,
+                            int T, int H, int tp_degree, float eps, tp_bf16* r_out,
+                            tp_bf16* n_out, tp_stream_t stream);
+
+/*
  * Largest activation h[T, F] (T * F * 2 bytes) that tp_mlp_forward_noalloc can
  * hold: 4 MiB, e.g. 64 tokens at F = 28672 or 2048 tokens at F = 1024.
  */

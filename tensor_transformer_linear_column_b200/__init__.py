@@ -47,6 +47,7 @@ SIGNATURES = {
     "tp_mlp_forward_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "tp_mlp_backward_workspace_bytes": (_Z, [_I, _I]),
     "tp_attn_decode_workspace_bytes": (_Z, [_I, _I, _I, _I, _I]),
+    "tp_sp_add_rmsnorm": (_I, [_P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "tp_attn_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
     "tp_mlp_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
                              _P]),
@@ -433,6 +434,27 @@ def tp_attn_decode(qkv: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "tp_attn_decode")
     return ctx
+
+
+def tp_sp_add_rmsnorm(y: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
+                      tp_degree: int, eps: float = 1e-5, r_out: Optional[torch.Tensor] = None,
+                      n_out: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None):
+    """(r, n): r = residual + y, n = RMSNorm(r) * gamma, by token shards of T / t."""
+    T, H = y.shape
+    if tuple(residual.shape) != (T, H) or tuple(gamma.shape) != (H,):
+        raise ValueError("residual must be [T, H] and gamma [H]")
+    dev = _device(y)
+    if r_out is None:
+        r_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    if n_out is None:
+        n_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    st = load().tp_sp_add_rmsnorm(_ptr(y, "y", dev), _ptr(residual, "residual", dev),
+                                  _ptr(gamma, "gamma", dev), T, H, int(tp_degree), float(eps),
+                                  _ptr(r_out, "r_out", dev), _ptr(n_out, "n_out", dev),
+                                  _stream(stream))
+    _check(st, "tp_sp_add_rmsnorm")
+    return r_out, n_out
 
 
 def tp_device_error_check() -> int:

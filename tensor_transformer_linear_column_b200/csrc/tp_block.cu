@@ -15,6 +15,7 @@
 #include "attn_kernel.cuh"
 #include "colsum_kernel.cuh"
 #include "diag_kernel.cuh"
+#include "norm_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "ptx.cuh"
 #include "stream_kernel.cuh"
@@ -855,6 +856,29 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
       return TP_ERR_CUDA;
   }
   return TP_OK;
+}
+
+tp_status tp_sp_add_rmsnorm(const tp_bf16* y, const tp_bf16* residual, const tp_bf16* gamma,
+                            int T, int H, int tp_degree, float eps, tp_bf16* r_out,
+                            tp_bf16* n_out, tp_stream_t stream) {
+  if (y == nullptr || residual == nullptr || gamma == nullptr || r_out == nullptr ||
+      n_out == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(y) || !aligned16(residual) || !aligned16(gamma) || !aligned16(r_out) ||
+      !aligned16(n_out))
+    return TP_ERR_ALIGN;
+  if (T < 1 || !feat_ok(H) || !(eps >= 0.0f)) return TP_ERR_SHAPE;
+  if (tp_degree < 1 || T % tp_degree != 0) return TP_ERR_TP_DEGREE;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(T), 1, 1);  // token shard s: rows [s T/t, (s+1) T/t)
+  cfg.blockDim = dim3(tpb::kNormThreads, 1, 1);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 0));
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tpb::add_rmsnorm_kernel, y, residual, gamma, H,
+                                           eps, r_out, n_out);
+  return cuda_ok(e, "launch add_rmsnorm_kernel") ? TP_OK : TP_ERR_CUDA;
 }
 
 tp_status tp_colpar_gemm_gelu_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scale,

@@ -202,6 +202,20 @@ def test_attn_decode_rejects_bad_arguments(lib):
         tp.TP_ERR_WORKSPACE
 
 
+def test_sp_norm_rejects_bad_arguments(lib):
+    def call(y=GOOD, g=GOOD, T=16, H=256, t=4, eps=1e-5, r=GOOD):
+        return lib.tp_sp_add_rmsnorm(y, GOOD, g, T, H, t, eps, r, GOOD, None)
+    assert call(y=None) == tp.TP_ERR_NULL
+    assert call(g=None) == tp.TP_ERR_NULL
+    assert call(r=ODD) == tp.TP_ERR_ALIGN
+    assert call(T=0) == tp.TP_ERR_SHAPE
+    assert call(H=100) == tp.TP_ERR_SHAPE
+    assert call(eps=-1.0) == tp.TP_ERR_SHAPE
+    assert call(eps=float("nan")) == tp.TP_ERR_SHAPE
+    assert call(t=3) == tp.TP_ERR_TP_DEGREE        # 16 tokens do not split 3 ways
+    assert call(t=0) == tp.TP_ERR_TP_DEGREE
+
+
 def test_attention_head_rules_from_the_pages(lib, golden):
     g = golden["head_divisibility"]
 
