@@ -55,11 +55,13 @@ KERNEL_SOURCES = {
     "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh"],
     "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh"],
     "attn_decode_kernel": ["csrc/ptx.cuh", "csrc/attn_kernel.cuh"],
+    "add_rmsnorm_kernel": ["csrc/ptx.cuh", "csrc/norm_kernel.cuh"],
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # default (timed steps, warm-up steps) per workload: about a second of timed work
 DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "attn70b_decode": (5000, 50),
+                 "sp405b": (2000, 20),
                  "mlp70b": (2000, 50),
                  "mlp70b_w8": (2000, 50), "sq4096": (20000, 200), "tiny": (20000, 200)}
 
@@ -269,6 +271,17 @@ class Workload:
             self.ws = torch.empty(max(tp.tp_attn_decode_workspace_bytes(
                 T, cfg.past, cfg.n_q_heads, cfg.n_kv_heads, d) for T in self.Ts),
                 dtype=torch.uint8, device=device)
+        elif name == "sp405b":
+            self.t = tp_degree or cfg.tp_degrees[0]
+            self.Ts = list(tokens or cfg.tokens)
+            ds = {T: workloads.sp_norm_inputs(cfg, T) for T in self.Ts}
+            self.xs = {T: d["y"] for T, d in ds.items()}
+            self.res = {T: d["residual"].to(device) for T, d in ds.items()}
+            self.weights = [ds[self.Ts[0]]["gamma"].to(device)]
+            self.weight_bytes = cfg.hidden * 2
+            self.hidden_in = self.hidden_out = cfg.hidden
+            self.r_out = {T: torch.empty((T, cfg.hidden), dtype=torch.bfloat16, device=device)
+                          for T in self.Ts}
         else:
             raise ValueError(name)
         self.xd = {T: x.to(device) for T, x in self.xs.items()}
@@ -276,7 +289,8 @@ class Workload:
                      for T in self.Ts}
         # rotate weight copies so each step reads weights evicted from L2
         assert self.weight_bytes == workload_weight_bytes(name)
-        self.rot = rotation_copies(self.weight_bytes) if rotate else 1
+        # (the sequence-parallel region streams activations only, all larger than L2)
+        self.rot = rotation_copies(self.weight_bytes) if rotate and name != "sp405b" else 1
         if self.rot > 1:
             base = self.weights[0]
             for _ in range(self.rot - 1):
@@ -285,7 +299,8 @@ class Workload:
                 else:
                     self.weights.append(base.clone())
         self.tokens_per_step = sum(self.Ts)
-        self.launches_per_step = len(self.Ts) * {"sq4096": 1, "attn70b_decode": 3}.get(name, 2)
+        self.launches_per_step = len(self.Ts) * {"sq4096": 1, "attn70b_decode": 3,
+                                                 "sp405b": 1}.get(name, 2)
 
     def step(self, i: int, xs=None, outs=None):
         tp = self.tp
@@ -300,6 +315,9 @@ class Workload:
             elif self.name == "mlp70b_w8":
                 tp.tp_mlp_forward_w8(xs[T], w[0], w[1], None, w[2], w[3], None, self.t,
                                      self.cfg.act, out=outs[T], workspace=self.ws)
+            elif self.name == "sp405b":
+                tp.tp_sp_add_rmsnorm(xs[T], self.res[T], w, self.t, 1e-5, r_out=self.r_out[T],
+                                     n_out=outs[T])
             elif self.name == "attn70b_decode":
                 c = self.cfg
                 tp.tp_attn_decode(xs[T], w[0], w[1], c.past, c.n_q_heads, c.n_kv_heads,
@@ -321,6 +339,8 @@ class Workload:
             if self.name == "attn70b_decode":
                 # the new tokens' keys and values: written to the cache, then read
                 b += 2 * 2 * 2 * T * self.cfg.n_kv_heads * self.cfg.head_dim
+            if self.name == "sp405b":
+                b += 2 * 2 * T * self.cfg.hidden  # the residual read and r written
             if self.name in ("tiny", "mlp70b", "mlp70b_w8", "mlp405b"):
                 b += 2 * 2 * T * self.cfg.ffn  # h written and read once
         return b
@@ -333,10 +353,13 @@ class Workload:
         return f
 
     def bound(self):
+        if self.name == "sp405b":
+            return "hbm"
         return "tensor" if max(self.Ts) > 256 else "hbm"
 
     def hbm_kernel(self):
-        return "attn_decode_kernel" if self.name == "attn70b_decode" else "stream_gemm_kernel"
+        return {"attn70b_decode": "attn_decode_kernel",
+                "sp405b": "add_rmsnorm_kernel"}.get(self.name, "stream_gemm_kernel")
 
 
 class _OracleRunner:
@@ -353,7 +376,14 @@ class _OracleRunner:
         cfg = workloads.CONFIGS[name]
         self.name = name
         self.cfg = cfg
-        if name == "attn70b_decode":
+        if name == "sp405b":
+            self.t = t or cfg.tp_degrees[0]
+            T0 = cfg.tokens[0]
+            d = workloads.sp_norm_inputs(cfg, T0)
+            rows = workloads.sample_rows(T0, 64)
+            self.y, self.res, self.gamma = d["y"][rows], d["residual"][rows], d["gamma"]
+            self.n_out = cfg.hidden
+        elif name == "attn70b_decode":
             self.t = t or cfg.tp_degrees[0]
             self.xs = {T: workloads.attn_decode_qkv(cfg, T) for T in cfg.tokens}
             self.k, self.v = workloads.attn_decode_cache(cfg)
@@ -392,11 +422,17 @@ class _OracleRunner:
         """Tokens a full oracle step covers (the sampled rows for prefill workloads)."""
         if self.name == "attn70b":
             return self.x.shape[0]
+        if self.name == "sp405b":
+            return self.y.shape[0]
         return sum(x.shape[0] for x in self.xs.values())
 
     def run(self, fraction, offset):
         """Compute the step on output-feature block [offset, offset + fraction * n_out)."""
         import oracle
+        if self.name == "sp405b":
+            # 64 seeded token rows (rows are independent); one token shard
+            oracle.sp_residual_norm([oracle.to_f64(self.y)], None, self.res, self.gamma, 1)
+            return 1.0
         if self.name == "attn70b_decode":
             # every new token needs the whole cache: the sample is whole calls
             c = self.cfg
@@ -507,6 +543,8 @@ def workload_weight_bytes(name):
         return 2 * cfg.hidden * cfg.ffn + 4 * (cfg.hidden + cfg.ffn)
     if name == "attn70b_decode":
         return 2 * cfg.n_kv_heads * cfg.past * cfg.head_dim * 2
+    if name == "sp405b":
+        return cfg.hidden * 2
     return 2 * cfg.hidden * cfg.ffn * 2
 
 
@@ -529,19 +567,26 @@ def workload_config(name, t, options, tokens=None):
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
         "attn70b_decode": "attention core decode, 64 query / 8 key-value heads of 128 (t=8), "
                           "65536 cached tokens, T=1,2,4 new tokens per call",
+        "sp405b": "sequence-parallel region of the 405B-shaped block: residual add + RMSNorm "
+                  "of T=8192 token rows of H=16384 in 8 token shards",
         "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192, column-parallel "
                    "up-projection + row-parallel down-projection with the fused 8-shard sum",
     }[name]
     wb = workload_weight_bytes(name)
-    rot = rotation_copies(wb)
+    rot = rotation_copies(wb) if name != "sp405b" else 1
     what = "KV caches" if name == "attn70b_decode" else "weights"
     if tokens:
         desc += f" (token counts overridden: {list(tokens)})"
+    if name == "sp405b":
+        l2 = (f"y, residual, r, n: {cfg.tokens[0] * cfg.hidden * 2 / 1e6:.0f} MB each > 126 MB "
+              f"L2, each read or written once per step")
+    else:
+        l2 = (f"{what} rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
+              f"the 126 MB L2): every call reads cold {what}" if rot > 1 else
+              f"{what} {wb / 1e6:.0f} MB > 126 MB L2, read once per step")
     return {"workload": desc, "name": name, "tp_degree": t, "tokens": list(tokens or cfg.tokens),
             "parallelism": "replicas (per-GPU block, t logical shards on chip)",
-            "l2": (f"{what} rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB >= 4x "
-                   f"the 126 MB L2): every call reads cold {what}" if rot > 1 else
-                   f"{what} {wb / 1e6:.0f} MB > 126 MB L2, read once per step"),
+            "l2": l2,
             "launch_options": options}
 
 

@@ -103,7 +103,9 @@ __global__ void kv_append_kernel(const uint16_t* __restrict__ qkv, uint16_t* __r
   grid_launch_dependents();
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
+// Two CTAs per SM (the ring of one overlaps the softmax of the other): at most
+// 170 registers per thread.
+__global__ void __launch_bounds__(kAttnThreads, 2)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
@@ -270,21 +272,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
     bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(s_bar), 0, abort_flag));
     tc_fence_after();
+    const int g_shift = __ffs(p.G) - 1;  // G is a power of two
     for (int c0 = 0; c0 < n_pad; c0 += 16) {
-      // pass 1: the chunk maximum of columns c0 .. c0 + 15 (masked scores -inf)
+      // the last key each of these 16 query rows may see (-1: a padding row)
+      int lim[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + ((c0 + j) >> g_shift);
+        lim[j] = tok < p.T ? p.past + tok : -1;
+      }
+      // pass 1: the chunk maximum of columns c0 .. c0 + 15 (masked scores
+      // -inf); two blocks' scores per TMEM round trip
       float mx[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) mx[j] = neg_inf();
-      for (int b = 0; ok && b < p.nb; ++b) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v);
+      for (int b = 0; ok && b < p.nb; b += 2) {
+        const bool two = b + 1 < p.nb;
+        uint32_t v0[16], v1[16];
+        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v0);
+        if (two) tmem_ld16(tmem + lane_addr + static_cast<uint32_t>((b + 1) * n_pad + c0), v1);
         tmem_wait_ld();
         const int key = key0 + b * kAttnBlockKeys + r;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int tok = tok0 + (c0 + j) / p.G;
-          const bool vis = tok < p.T && key <= p.past + tok;
-          if (vis) mx[j] = fmaxf(mx[j], __uint_as_float(v[j]) * p.scale_log2);
+          if (key <= lim[j]) mx[j] = fmaxf(mx[j], __uint_as_float(v0[j]) * p.scale_log2);
+          if (two && key + kAttnBlockKeys <= lim[j])
+            mx[j] = fmaxf(mx[j], __uint_as_float(v1[j]) * p.scale_log2);
         }
       }
 #pragma unroll
@@ -313,24 +326,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float sum[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) sum[j] = 0.0f;
-      for (int b = 0; ok && b < p.nb; ++b) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v);
+      // P_b half (key / 64), row n: 128-byte rows, 16-byte chunk (key % 64) / 8
+      // stored at chunk ^ (n % 8)
+      const int kc = (r & 63) >> 3, kw = (r & 7) * 2;
+      for (int b = 0; ok && b < p.nb; b += 2) {
+        const bool two = b + 1 < p.nb;
+        uint32_t v0[16], v1[16];
+        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v0);
+        if (two) tmem_ld16(tmem + lane_addr + static_cast<uint32_t>((b + 1) * n_pad + c0), v1);
         tmem_wait_ld();
-        const int key = key0 + b * kAttnBlockKeys + r;
-        // P_b half (key / 64), row n: 128-byte rows, 16-byte chunk (key % 64) / 8
-        // stored at chunk ^ (n % 8)
-        uint8_t* pb = ps + static_cast<size_t>(b) * 2u * q_half + static_cast<size_t>(r >> 6) * q_half;
-        const int kc = (r & 63) >> 3, kw = (r & 7) * 2;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = c0 + j;
-          const int tok = tok0 + n / p.G;
-          const bool vis = tok < p.T && key <= p.past + tok;
-          const float e = vis ? exp2f(__uint_as_float(v[j]) * p.scale_log2 - msafe[j]) : 0.0f;
-          const __nv_bfloat16 hb = __float2bfloat16_rn(e);
-          sum[j] += __bfloat162float(hb);
-          *reinterpret_cast<__nv_bfloat16*>(pb + n * 128 + ((kc ^ (n & 7)) << 4) + kw) = hb;
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          const int bb = b + h;
+          const int key = key0 + bb * kAttnBlockKeys + r;
+          uint8_t* pb = ps + static_cast<size_t>(bb) * 2u * q_half + static_cast<size_t>(r >> 6) * q_half;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            const float sv = __uint_as_float(h == 0 ? v0[j] : v1[j]);
+            const float e = key <= lim[j] ? exp2f(sv * p.scale_log2 - msafe[j]) : 0.0f;
+            const __nv_bfloat16 hb = __float2bfloat16_rn(e);
+            sum[j] += __bfloat162float(hb);
+            *reinterpret_cast<__nv_bfloat16*>(pb + n * 128 + ((kc ^ (n & 7)) << 4) + kw) = hb;
+          }
         }
       }
 #pragma unroll

@@ -571,11 +571,21 @@ tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& g
   }
   p.n_pad = p.Tq * G;
   const int nblk = (p.L + tpb::kAttnBlockKeys - 1) / tpb::kAttnBlockKeys;
-  // S of every block of a chunk plus O in at most 256 TMEM columns
-  int nb_max = 256 / p.n_pad - 1;
-  nb_max = nb_max < 1 ? 1 : (nb_max > 8 ? 8 : nb_max);
-  int nb = (nkv * groups * nblk + kAttnTargetCtas - 1) / kAttnTargetCtas;
-  nb = nb < 1 ? 1 : (nb > nb_max ? nb_max : nb);
+  // S of every block of a chunk plus O in at most 256 TMEM columns, and the
+  // chunk's P small enough that two CTAs share an SM: 8 blocks at 16 query
+  // rows, 4 at 32
+  const int nb_max = p.n_pad <= 16 ? 8 : 4;
+  // the fewest chunks (largest nb) whose grid fills whole waves of
+  // kAttnTargetCtas CTAs, so no wave runs part-empty
+  const int per_chunk = nkv * groups;  // CTAs per chunk index
+  int nb = nb_max;
+  for (int cand = nb_max; cand >= 1; --cand) {
+    const int ctas = per_chunk * ((nblk + cand - 1) / cand);
+    if (ctas % kAttnTargetCtas == 0 || ctas * 4 >= 3 * kAttnTargetCtas * ((ctas + kAttnTargetCtas - 1) / kAttnTargetCtas)) {
+      nb = cand;
+      break;
+    }
+  }
   p.nb = nb;
   p.chunks = (nblk + nb - 1) / nb;
   p.tmem_cols = next_pow2((nb + 1) * p.n_pad < 32 ? 32 : (nb + 1) * p.n_pad);

@@ -144,6 +144,16 @@ class AttnDecodeConfig:
     tp_degrees: Tuple[int, ...]
 
 
+@dataclasses.dataclass(frozen=True)
+class SPNormConfig:
+    """The sequence-parallel region after a row-parallel linear: residual add
+    and RMSNorm of every token row, by token shards."""
+    name: str
+    hidden: int
+    tokens: Tuple[int, ...]
+    tp_degrees: Tuple[int, ...]
+
+
 CONFIGS: Dict[str, object] = {
     # x[8,256] fp32, W1[256->1024], W2[1024->256] N(0,0.02), biases N(0,0.01), t=2
     "tiny": MLPConfig("tiny", hidden=256, ffn=1024, tokens=(8,), tp_degrees=(2,),
@@ -166,6 +176,8 @@ CONFIGS: Dict[str, object] = {
     "attn70b_decode": AttnDecodeConfig("attn70b_decode", n_q_heads=64, n_kv_heads=8,
                                        head_dim=128, past=65536, tokens=(1, 2, 4),
                                        tp_degrees=(8,)),
+    # the sequence-parallel region of the 405B-shaped block in prefill
+    "sp405b": SPNormConfig("sp405b", hidden=16384, tokens=(8192,), tp_degrees=(8,)),
     # 405B-shaped MLP prefill; the oracle checks 64 seeded rows
     "mlp405b": MLPConfig("mlp405b", hidden=16384, ffn=53248, tokens=(8192,),
                          tp_degrees=(8,), act="gelu_tanh", w_std=0.01, b_std=None,
@@ -240,6 +252,15 @@ def attn_decode_cache(cfg: AttnDecodeConfig, seed: int = 0) -> Tuple[torch.Tenso
     """The caches k, v [nkv, past, d] of the cached tokens, N(0, 1) bf16."""
     shape = (cfg.n_kv_heads, cfg.past, cfg.head_dim)
     return normal_bf16(shape, 1.0, seed, 601), normal_bf16(shape, 1.0, seed, 602)
+
+
+def sp_norm_inputs(cfg: SPNormConfig, T: int, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """y (the row-parallel output) and the residual [T, H] ~ N(0, 1), and
+    gamma [H] ~ 1 + N(0, 0.1^2), bf16."""
+    y = normal_bf16((T, cfg.hidden), 1.0, seed, 700 + int(T))
+    res = normal_bf16((T, cfg.hidden), 1.0, seed, 800 + int(T))
+    gamma = (1.0 + normal_bf16((cfg.hidden,), 0.1, seed, 701).float()).to(torch.bfloat16)
+    return {"y": y, "residual": res, "gamma": gamma}
 
 
 def quantize_e4m3_rows(w: torch.Tensor, rows_per_chunk: int = 2048
