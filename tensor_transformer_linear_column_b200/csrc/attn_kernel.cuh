@@ -21,21 +21,24 @@
 //   attn_combine_kernel   per (token, query head): the partials of all chunks
 //                         merged in chunk order, divided by the total sum.
 //
-// attn_decode_kernel, per CTA (one M = 128 key block = 32 KB of K or V per
-// ring stage, loaded by TMA):
-//   S^T[key, n] = K_blk Q^T    tcgen05.mma, keys as M, the N = G Tq query rows
-//                              (token-major, head-minor) as N, d = 128 as K;
-//                              every block of the chunk into its own TMEM slice
-//   softmax                    the four epilogue warps (one key per thread)
-//                              mask, take the chunk maximum per query row,
-//                              p = 2^(s - m) rounded to bf16 into shared memory
-//                              as the next MMA's K-major B operand, sum l
-//   O^T[d, n] += V_blk^T P^T   tcgen05.mma, d as M: V is read MN-major straight
+// attn_decode_kernel, per CTA (blocks of 128 keys; a 32 KB ring stage holds
+// one block of K or of V, loaded by TMA in the order K_0, K_1, V_0, K_2, V_1, ...):
+//   S_b^T[key, n] = K_b Q^T    tcgen05.mma, keys as M, the N = G Tq query rows
+//                              (token-major, head-minor) as N, d = 128 as K, into
+//                              one of two TMEM score slots
+//   softmax of block b         the four epilogue warps (one key per thread):
+//                              mask, the block maximum per query row, the
+//                              running maximum m, p = 2^(s - m) rounded to bf16
+//                              into one of two shared-memory P slots (the next
+//                              MMA's K-major B operand), the running sum l
+//                              rescaled by alpha = 2^(m_old - m), and the
+//                              accumulator O rescaled by alpha in TMEM
+//   O^T[d, n] += V_b^T P_b^T   tcgen05.mma, d as M: V is read MN-major straight
 //                              from its [key][d] tile, keys as K
-// Because the maximum over the whole chunk is known before any P V product,
-// no accumulator is ever rescaled.  HBM traffic is the cache read once per
-// token group (K and V, 512 bytes per key at d = 128) plus partials of
-// (d + 2) * 4 bytes per query row per chunk.
+// The scores of block b + 1 are computed while block b's softmax runs, and
+// block b's P V product while block b + 1's scores are read.  HBM traffic is
+// the cache read once per token group (K and V, 512 bytes per key at d = 128)
+// plus partials of (d + 2) * 4 bytes per query row per chunk.
 #pragma once
 
 #include "ptx.cuh"
@@ -44,7 +47,7 @@ namespace tpb {
 
 constexpr int kAttnHeadDim = 128;
 constexpr int kAttnBlockKeys = 128;
-constexpr int kAttnStages = 2;
+constexpr int kAttnMaxStages = 3;
 constexpr int kAttnThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue
 constexpr int kAttnBlockBytes = kAttnBlockKeys * kAttnHeadDim * 2;  // 32 KB
 constexpr int kAttnHalfBytes = kAttnBlockBytes / 2;                // one 64-wide d half
@@ -57,24 +60,23 @@ struct AttnParams {
   int nq, nkv, G; // query heads, key-value heads, G = nq / nkv
   int Tq;         // tokens per token group (grid z)
   int n_pad;      // query rows per CTA: G * Tq, 16 or 32
-  int nb;         // key blocks per chunk
+  int nblk;       // key blocks of 128 in [0, L)
+  int nb;         // key blocks per chunk (the last chunk may have fewer)
   int chunks;     // chunks per key-value head
+  int stages;     // ring depth
   int tmem_cols;  // TMEM columns allocated (power of two)
   float scale_log2;  // log2(e) / sqrt(d)
   float* part_o;  // [groups][nkv][chunks][n_pad][d] unnormalised sums of p v
   float* part_ml; // [groups][nkv][chunks][n_pad][2]  (max m, sum l) in base-2 units
 };
 
-// Shared memory (dynamic, base rounded up to 1024 B): ring [kAttnStages][32 KB],
-// Q [2 halves][n_pad][64] bf16, P [nb][2 halves][n_pad][64] bf16, reduction
-// scratch [4][16] floats, m / l [n_pad] floats, barriers.
+// Shared memory (dynamic, base rounded up to 1024 B): ring [stages][32 KB],
+// Q [2 d halves][n_pad][64] bf16, P [2 slots][2 key halves][n_pad][64] bf16,
+// reduction scratch [2][4][32] floats, m / l / alpha [32] floats, barriers.
 __host__ __device__ inline int attn_q_bytes(int n_pad) { return n_pad * kAttnHeadDim * 2; }
-__host__ __device__ inline int attn_p_bytes(int nb, int n_pad) {
-  return nb * n_pad * kAttnBlockKeys * 2;
-}
-__host__ __device__ inline int attn_smem_bytes(int nb, int n_pad) {
-  return 1024 + kAttnStages * kAttnBlockBytes + attn_q_bytes(n_pad) + attn_p_bytes(nb, n_pad) +
-         4 * 16 * 4 + 2 * n_pad * 4 + (2 * kAttnStages + 5) * 8 + 16;
+__host__ __device__ inline int attn_smem_bytes(int stages, int n_pad) {
+  return 1024 + stages * kAttnBlockBytes + 3 * attn_q_bytes(n_pad) + 2 * 4 * 32 * 4 + 3 * 32 * 4 +
+         (2 * kAttnMaxStages + 10) * 8 + 16;
 }
 
 // Copy the new tokens' keys and values into the cache: for token i and
@@ -104,7 +106,8 @@ __global__ void kv_append_kernel(const uint16_t* __restrict__ qkv, uint16_t* __r
 }
 
 // Two CTAs per SM (the ring of one overlaps the softmax of the other): at most
-// 170 registers per thread.
+// 170 registers per thread.  kRows = n_pad (16 or 32).
+template <int kRows>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
@@ -112,20 +115,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t kQHalf = kRows * 128u;  // bytes of one 64-wide half of a [kRows][128] tile
   uint8_t* ring = smem;
-  uint8_t* qs = ring + kAttnStages * kAttnBlockBytes;
-  uint8_t* ps = qs + attn_q_bytes(p.n_pad);
-  float* red = reinterpret_cast<float*>(ps + attn_p_bytes(p.nb, p.n_pad));  // [4][16]
-  float* m_s = red + 4 * 16;                                                 // [n_pad]
-  float* l_s = m_s + p.n_pad;                                                // [n_pad]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(l_s + p.n_pad);
-  uint64_t* full_bar = bars;                       // [stages]
-  uint64_t* empty_bar = bars + kAttnStages;        // [stages]
-  uint64_t* q_bar = bars + 2 * kAttnStages;
-  uint64_t* s_bar = q_bar + 1;                     // every S block is in TMEM
-  uint64_t* p_bar = q_bar + 2;                     // P is in shared memory (128 arrivals)
-  uint64_t* o_bar = q_bar + 3;                     // O is in TMEM
-  uint64_t* final_bar = q_bar + 4;
+  uint8_t* qs = ring + p.stages * kAttnBlockBytes;
+  uint8_t* ps = qs + 2 * kQHalf;                          // [2 slots][2 halves][kRows][128 B]
+  float* red_m = reinterpret_cast<float*>(ps + 4 * kQHalf);  // [4][32]
+  float* red_s = red_m + 4 * 32;                             // [4][32]
+  float* m_s = red_s + 4 * 32;                               // [32] running maximum
+  float* l_s = m_s + 32;                                     // [32] running sum
+  float* a_s = l_s + 32;                                     // [32] this block's alpha
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + 32);
+  uint64_t* full_bar = bars;                         // [kAttnMaxStages]
+  uint64_t* empty_bar = bars + kAttnMaxStages;       // [kAttnMaxStages]
+  uint64_t* q_bar = bars + 2 * kAttnMaxStages;
+  uint64_t* s_full = q_bar + 1;                      // [2] scores of a block in TMEM slot
+  uint64_t* s_free = q_bar + 3;                      // [2] slot read by the softmax (128)
+  uint64_t* p_full = q_bar + 5;                      // [2] P slot written, O rescaled (128)
+  uint64_t* o_done = q_bar + 7;                      // [2] the P V product of the slot done
+  uint64_t* final_bar = q_bar + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -134,20 +141,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int chunk = blockIdx.x;
   const int g = blockIdx.y;
   const int grp = blockIdx.z;
-  const int key0 = chunk * p.nb * kAttnBlockKeys;
+  const int blk0 = chunk * p.nb;
+  const int nbc = p.nblk - blk0 < p.nb ? p.nblk - blk0 : p.nb;  // blocks of this chunk
+  const int key0 = blk0 * kAttnBlockKeys;
   const int tok0 = grp * p.Tq;
-  const int n_pad = p.n_pad;
-  const uint32_t q_half = static_cast<uint32_t>(n_pad) * 128u;  // bytes of one d half of Q
+  const int nload = 2 * nbc;
+  const int stages = p.stages;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAttnStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     mbar_init(smem_u32(q_bar), 1);
-    mbar_init(smem_u32(s_bar), 1);
-    mbar_init(smem_u32(p_bar), 128);
-    mbar_init(smem_u32(o_bar), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), 128);
+      mbar_init(smem_u32(&p_full[i]), 128);
+      mbar_init(smem_u32(&o_done[i]), 1);
+    }
     mbar_init(smem_u32(final_bar), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -159,42 +171,52 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int nload = 2 * p.nb;  // K blocks, then V blocks
+  const uint32_t tmem = *tmem_slot;   // S slots at columns 0 and kRows, O at 2 kRows
+  const uint32_t o_col = 2u * kRows;
+
+  // load / MMA item i: K_0, then K_b, V_{b-1} for b = 1 .. nbc-1, then V_{nbc-1}
+  auto item = [nload](int i, bool& is_v) -> int {
+    if (i == 0) { is_v = false; return 0; }
+    if (i == nload - 1) { is_v = true; return (nload >> 1) - 1; }
+    is_v = (i & 1) == 0;
+    return is_v ? (i >> 1) - 1 : (i + 1) >> 1;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: Q once, then K_0 .. K_nb-1, V_0 .. V_nb-1
+      // ---------------- TMA producer
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
       grid_dependency_wait();  // qkv and the appended cache rows come from preceding kernels
       const uint32_t qb = smem_u32(q_bar);
-      mbar_arrive_expect_tx(qb, 2u * q_half);
+      mbar_arrive_expect_tx(qb, 2u * kQHalf);
       tma_load_3d(smem_u32(qs), &tmap_q, qb, 0, g * p.G, tok0);
-      tma_load_3d(smem_u32(qs) + q_half, &tmap_q, qb, 64, g * p.G, tok0);
+      tma_load_3d(smem_u32(qs) + kQHalf, &tmap_q, qb, 64, g * p.G, tok0);
       uint32_t issued = 0u, phases = 0u;
       int s = 0;
       uint32_t ph = 0u;
       for (int i = 0; i < nload; ++i) {
         if (!wait_parity(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag)) break;
+        bool is_v;
+        const int b = item(i, is_v);
         const uint32_t fb = smem_u32(&full_bar[s]);
         const uint32_t dst = smem_u32(ring + s * kAttnBlockBytes);
-        const CUtensorMap* map = i < p.nb ? &tmap_k : &tmap_v;
-        const int kb = key0 + (i < p.nb ? i : i - p.nb) * kAttnBlockKeys;
+        const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+        const int kb = key0 + b * kAttnBlockKeys;
         mbar_arrive_expect_tx(fb, kAttnBlockBytes);
         tma_load_3d(dst, map, fb, 0, kb, g);
         tma_load_3d(dst + kAttnHalfBytes, map, fb, 64, kb, g);
         issued |= 1u << s;
         phases = (phases & ~(1u << s)) | (ph << s);
-        if (++s == kAttnStages) {
+        if (++s == stages) {
           s = 0;
           ph ^= 1u;
         }
       }
       if (*abort_flag) {
         drain_wait(qb, 0, 50ull * 1000ull * 1000ull);
-        for (int st = 0; st < kAttnStages; ++st)
+        for (int st = 0; st < stages; ++st)
           if (issued & (1u << st))
             drain_wait(smem_u32(&full_bar[st]), (phases >> st) & 1u, 50ull * 1000ull * 1000ull);
       }
@@ -202,23 +224,29 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
-      const uint32_t idesc_s = idesc_bf16_f32(128, n_pad);               // K, Q both K-major
-      const uint32_t idesc_o = idesc_bf16_f32(128, n_pad, true, false);  // V^T MN-major, P K-major
-      const uint32_t o_col = static_cast<uint32_t>(p.nb * n_pad);
+      // ---------------- MMA issuer, same item order as the loads
+      const uint32_t idesc_s = idesc_bf16_f32(128, kRows);               // K, Q both K-major
+      const uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, false);  // V^T MN-major, P K-major
       bool ok = wait_parity(smem_u32(q_bar), 0, abort_flag);
       tc_fence_after();
       int s = 0;
       uint32_t ph = 0u;
       for (int i = 0; ok && i < nload; ++i) {
-        if (i == p.nb) {
-          // all S blocks issued: tell the softmax warps, then wait for P
-          umma_commit(smem_u32(s_bar));
-          if (!wait_parity(smem_u32(p_bar), 0, abort_flag)) {
+        bool is_v;
+        const int b = item(i, is_v);
+        const int slot = b & 1;
+        if (!is_v) {
+          // the score slot must have been read by the softmax of block b - 2
+          if (b >= 2 && !wait_parity(smem_u32(&s_free[slot]), ((b - 2) >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
+        } else {
+          // P_b written and O rescaled for block b
+          if (!wait_parity(smem_u32(&p_full[slot]), (b >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
         }
         if (!wait_parity(smem_u32(&full_bar[s]), ph, abort_flag)) {
           ok = false;
@@ -226,165 +254,173 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
         tc_fence_after();
         const uint32_t st = smem_u32(ring + s * kAttnBlockBytes);
-        if (i < p.nb) {
+        if (!is_v) {
           // S_b^T = K_b Q^T, K = d in steps of 16: steps 0-3 in d half 0, 4-7 in half 1
-          const uint32_t d = tmem + static_cast<uint32_t>(i * n_pad);
+          const uint32_t d = tmem + static_cast<uint32_t>(slot * kRows);
 #pragma unroll
           for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
             const uint32_t hk = static_cast<uint32_t>(kk >> 2), ck = static_cast<uint32_t>(kk & 3);
             umma_bf16(d, desc_kmajor_sw128(st + hk * kAttnHalfBytes + ck * 32u),
-                      desc_kmajor_sw128(smem_u32(qs) + hk * q_half + ck * 32u), idesc_s,
+                      desc_kmajor_sw128(smem_u32(qs) + hk * kQHalf + ck * 32u), idesc_s,
                       kk > 0 ? 1u : 0u);
           }
+          umma_commit(smem_u32(&empty_bar[s]));
+          umma_commit(smem_u32(&s_full[slot]));
         } else {
           // O^T += V_b^T P_b^T, K = keys in steps of 16: V MN-major (d halves
-          // 16 KB apart, 8-key groups 1024 B apart); P_b's two 64-key halves
-          const int b = i - p.nb;
-          const uint32_t pb = smem_u32(ps) + static_cast<uint32_t>(b) * 2u * q_half;
+          // 16 KB apart, 8-key groups 1024 B apart); P slot's two 64-key halves
+          const uint32_t pb = smem_u32(ps) + static_cast<uint32_t>(slot) * 2u * kQHalf;
 #pragma unroll
           for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk) {
             const uint32_t hk = static_cast<uint32_t>(kk >> 2), ck = static_cast<uint32_t>(kk & 3);
             umma_bf16(tmem + o_col,
                       desc_mnmajor_sw128(st + static_cast<uint32_t>(kk) * 2048u, kAttnHalfBytes),
-                      desc_kmajor_sw128(pb + hk * q_half + ck * 32u), idesc_o,
+                      desc_kmajor_sw128(pb + hk * kQHalf + ck * 32u), idesc_o,
                       (b > 0 || kk > 0) ? 1u : 0u);
           }
+          umma_commit(smem_u32(&empty_bar[s]));
+          umma_commit(smem_u32(&o_done[slot]));
         }
-        umma_commit(smem_u32(&empty_bar[s]));
-        if (++s == kAttnStages) {
+        if (++s == stages) {
           s = 0;
           ph ^= 1u;
         }
       }
-      if (ok) umma_commit(smem_u32(o_bar));
       // every MMA issued by this thread is complete once final_bar flips
       umma_commit(smem_u32(final_bar));
       drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
     }
     __syncwarp();
   } else {
-    // ---------------- warps 2-5: softmax and the partial's write-out.
-    // Thread r of the 128 owns TMEM lane r: key r of each block, then d = r.
+    // ---------------- warps 2-5: softmax per block, O rescale, the partial.
+    // Thread r of the 128 owns TMEM lane r: key r of each block, and d = r of O.
+    // Every thread takes the same named barriers and arrivals whatever its
+    // waits returned, so a timed-out wait cannot leave a barrier short.
     grid_dependency_wait();  // the partial buffers may still be read by a preceding kernel
-    const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+    const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
-    const int et = threadIdx.x - 64;         // 0..127, for shared-memory roles
+    const int et = threadIdx.x - 64;  // 0..127
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    bool ok = __all_sync(0xffffffffu, wait_parity(smem_u32(s_bar), 0, abort_flag));
-    tc_fence_after();
     const int g_shift = __ffs(p.G) - 1;  // G is a power of two
-    for (int c0 = 0; c0 < n_pad; c0 += 16) {
-      // the last key each of these 16 query rows may see (-1: a padding row)
-      int lim[16];
+    int lim[kRows];                      // last key each query row may see (-1: padding)
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int tok = tok0 + ((c0 + j) >> g_shift);
-        lim[j] = tok < p.T ? p.past + tok : -1;
-      }
-      // pass 1: the chunk maximum of columns c0 .. c0 + 15 (masked scores
-      // -inf); two blocks' scores per TMEM round trip
-      float mx[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) mx[j] = neg_inf();
-      for (int b = 0; ok && b < p.nb; b += 2) {
-        const bool two = b + 1 < p.nb;
-        uint32_t v0[16], v1[16];
-        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v0);
-        if (two) tmem_ld16(tmem + lane_addr + static_cast<uint32_t>((b + 1) * n_pad + c0), v1);
-        tmem_wait_ld();
-        const int key = key0 + b * kAttnBlockKeys + r;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (key <= lim[j]) mx[j] = fmaxf(mx[j], __uint_as_float(v0[j]) * p.scale_log2);
-          if (two && key + kAttnBlockKeys <= lim[j])
-            mx[j] = fmaxf(mx[j], __uint_as_float(v1[j]) * p.scale_log2);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], o));
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) red[q4 * 16 + j] = mx[j];
-      }
-      named_barrier_sync(1, 128);
-      if (et < 16) {
-        const float m = fmaxf(fmaxf(red[et], red[16 + et]), fmaxf(red[32 + et], red[48 + et]));
-        m_s[c0 + et] = m;
-      }
-      named_barrier_sync(1, 128);
-      float msafe[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float m = m_s[c0 + j];
-        msafe[j] = m == neg_inf() ? 0.0f : m;  // a row with nothing visible: p = 0
-      }
-      // pass 2: p = 2^(s - m) as bf16 into P (row n = column of S, key r of the
-      // block), and the sum of the rounded p of each row
-      float sum[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) sum[j] = 0.0f;
-      // P_b half (key / 64), row n: 128-byte rows, 16-byte chunk (key % 64) / 8
-      // stored at chunk ^ (n % 8)
-      const int kc = (r & 63) >> 3, kw = (r & 7) * 2;
-      for (int b = 0; ok && b < p.nb; b += 2) {
-        const bool two = b + 1 < p.nb;
-        uint32_t v0[16], v1[16];
-        tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(b * n_pad + c0), v0);
-        if (two) tmem_ld16(tmem + lane_addr + static_cast<uint32_t>((b + 1) * n_pad + c0), v1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h == 1 && !two) break;
-          const int bb = b + h;
-          const int key = key0 + bb * kAttnBlockKeys + r;
-          uint8_t* pb = ps + static_cast<size_t>(bb) * 2u * q_half + static_cast<size_t>(r >> 6) * q_half;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            const float sv = __uint_as_float(h == 0 ? v0[j] : v1[j]);
-            const float e = key <= lim[j] ? exp2f(sv * p.scale_log2 - msafe[j]) : 0.0f;
-            const __nv_bfloat16 hb = __float2bfloat16_rn(e);
-            sum[j] += __bfloat162float(hb);
-            *reinterpret_cast<__nv_bfloat16*>(pb + n * 128 + ((kc ^ (n & 7)) << 4) + kw) = hb;
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum[j] += __shfl_xor_sync(0xffffffffu, sum[j], o);
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) red[q4 * 16 + j] = sum[j];
-      }
-      named_barrier_sync(1, 128);
-      if (et < 16) l_s[c0 + et] = ((red[et] + red[16 + et]) + red[32 + et]) + red[48 + et];
-      named_barrier_sync(1, 128);
+    for (int j = 0; j < kRows; ++j) {
+      const int tok = tok0 + (j >> g_shift);
+      lim[j] = tok < p.T ? p.past + tok : -1;
     }
-    // P is complete: make the generic-proxy writes visible to the MMA
-    fence_proxy_async_smem();
-    tc_fence_before();
-    mbar_arrive(smem_u32(p_bar));
-    ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(o_bar), 0, abort_flag));
+    if (et < kRows) {
+      m_s[et] = neg_inf();
+      l_s[et] = 0.0f;
+    }
+    // P half (key / 64) of row n: 128-byte rows, 16-byte chunk (key % 64) / 8
+    // stored at chunk ^ (n % 8)
+    const int kc = (r & 63) >> 3, kw = (r & 7) * 2;
+    bool ok = true;
+    for (int b = 0; b < nbc; ++b) {
+      const int slot = b & 1;
+      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&s_full[slot]), (b >> 1) & 1,
+                                                     abort_flag));
+      tc_fence_after();
+      uint32_t v[kRows];
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < kRows; c += 16)
+          tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(slot * kRows + c),
+                    *reinterpret_cast<uint32_t(*)[16]>(v + c));
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) v[j] = 0u;
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[slot]));
+      const int key = key0 + b * kAttnBlockKeys + r;
+      float sc[kRows];
+#pragma unroll
+      for (int j = 0; j < kRows; ++j)
+        sc[j] = key <= lim[j] ? __uint_as_float(v[j]) * p.scale_log2 : neg_inf();
+      // the block maximum per row: warp butterfly, then the four warps
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        float mx = sc[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) red_m[q4 * 32 + j] = mx;
+      }
+      named_barrier_sync(1, 128);
+      if (et < kRows) {
+        const float mb = fmaxf(fmaxf(red_m[et], red_m[32 + et]), fmaxf(red_m[64 + et], red_m[96 + et]));
+        const float mo = m_s[et];
+        const float mn = fmaxf(mo, mb);
+        a_s[et] = mo == neg_inf() ? 0.0f : exp2f(mo - mn);
+        m_s[et] = mn;
+      }
+      named_barrier_sync(1, 128);
+      // the P slot is free once the P V product of block b - 2 is done
+      if (b >= 2)
+        ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[slot]),
+                                                       ((b - 2) >> 1) & 1, abort_flag));
+      uint8_t* pslot = ps + static_cast<size_t>(slot) * 2u * kQHalf + static_cast<size_t>(r >> 6) * kQHalf;
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        const float m = m_s[j];
+        const float e = sc[j] == neg_inf() ? 0.0f : exp2f(sc[j] - m);
+        const __nv_bfloat16 hb = __float2bfloat16_rn(e);
+        *reinterpret_cast<__nv_bfloat16*>(pslot + j * 128 + ((kc ^ (j & 7)) << 4) + kw) = hb;
+        float sm = __bfloat162float(hb);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        if (lane == 0) red_s[q4 * 32 + j] = sm;
+      }
+      named_barrier_sync(1, 128);
+      if (et < kRows)
+        l_s[et] = fmaf(l_s[et], a_s[et],
+                       ((red_s[et] + red_s[32 + et]) + red_s[64 + et]) + red_s[96 + et]);
+      // O (the P V products of blocks < b) times alpha, once block b - 1's is done
+      if (b >= 1) {
+        ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[(b - 1) & 1]),
+                                                       ((b - 1) >> 1) & 1, abort_flag));
+        tc_fence_after();
+        if (ok) {
+          uint32_t o[kRows];
+#pragma unroll
+          for (int c = 0; c < kRows; c += 16)
+            tmem_ld16(tmem + lane_addr + o_col + static_cast<uint32_t>(c),
+                      *reinterpret_cast<uint32_t(*)[16]>(o + c));
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < kRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a_s[j]);
+#pragma unroll
+          for (int c = 0; c < kRows; c += 16)
+            tmem_st16(tmem + lane_addr + o_col + static_cast<uint32_t>(c),
+                      *reinterpret_cast<uint32_t(*)[16]>(o + c));
+          tmem_wait_st();
+        }
+      }
+      fence_proxy_async_smem();  // P is read by the MMA through the async proxy
+      tc_fence_before();
+      mbar_arrive(smem_u32(&p_full[slot]));
+    }
+    // the last P V product, then the partial: O^T (lane = d, column = query row)
+    if (nbc > 0)
+      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[(nbc - 1) & 1]),
+                                                     ((nbc - 1) >> 1) & 1, abort_flag));
     tc_fence_after();
-    // O^T in TMEM: lane = d, column = query row n.  Partial of (chunk, head g,
-    // group): part_o[.., n, d] (coalesced over d), part_ml[.., n] = (m, l)
     const size_t slot = (static_cast<size_t>(grp) * p.nkv + g) * p.chunks + chunk;
-    float* po = p.part_o + slot * static_cast<size_t>(n_pad) * kAttnHeadDim;
-    for (int c0 = 0; c0 < n_pad; c0 += 16) {
+    float* po = p.part_o + slot * static_cast<size_t>(kRows) * kAttnHeadDim;
+#pragma unroll
+    for (int c = 0; c < kRows; c += 16) {
       uint32_t v[16];
-      tmem_ld16(tmem + lane_addr + static_cast<uint32_t>(p.nb * n_pad + c0), v);
-      tmem_wait_ld();
+      if (ok) {
+        tmem_ld16(tmem + lane_addr + o_col + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+      }
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        po[static_cast<size_t>(c0 + j) * kAttnHeadDim + r] = ok ? __uint_as_float(v[j]) : 0.0f;
+        po[static_cast<size_t>(c + j) * kAttnHeadDim + r] = ok ? __uint_as_float(v[j]) : 0.0f;
     }
-    if (et < n_pad) {
-      float* pml = p.part_ml + slot * static_cast<size_t>(n_pad) * 2;
+    if (et < kRows) {
+      float* pml = p.part_ml + slot * static_cast<size_t>(kRows) * 2;
       pml[2 * et] = ok ? m_s[et] : neg_inf();
       pml[2 * et + 1] = ok ? l_s[et] : 0.0f;
     }

@@ -134,7 +134,10 @@ const DeviceInfo* device_info() {
                                       tpb::kPairSmemBytes),
                  "cudaFuncSetAttribute"))
       return nullptr;
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_decode_kernel,
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_decode_kernel<16>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::attn_decode_kernel<32>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                "cudaFuncSetAttribute"))
     return nullptr;
@@ -570,25 +573,18 @@ tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& g
     groups = (T + tq_max - 1) / tq_max;
   }
   p.n_pad = p.Tq * G;
-  const int nblk = (p.L + tpb::kAttnBlockKeys - 1) / tpb::kAttnBlockKeys;
-  // S of every block of a chunk plus O in at most 256 TMEM columns, and the
-  // chunk's P small enough that two CTAs share an SM: 8 blocks at 16 query
-  // rows, 4 at 32
-  const int nb_max = p.n_pad <= 16 ? 8 : 4;
-  // the fewest chunks (largest nb) whose grid fills whole waves of
-  // kAttnTargetCtas CTAs, so no wave runs part-empty
+  p.nblk = (p.L + tpb::kAttnBlockKeys - 1) / tpb::kAttnBlockKeys;
+  // chunks per key-value head so the grid is about kAttnTargetCtas CTAs (two
+  // per SM, one wave); every chunk streams nb blocks with a running softmax
   const int per_chunk = nkv * groups;  // CTAs per chunk index
-  int nb = nb_max;
-  for (int cand = nb_max; cand >= 1; --cand) {
-    const int ctas = per_chunk * ((nblk + cand - 1) / cand);
-    if (ctas % kAttnTargetCtas == 0 || ctas * 4 >= 3 * kAttnTargetCtas * ((ctas + kAttnTargetCtas - 1) / kAttnTargetCtas)) {
-      nb = cand;
-      break;
-    }
-  }
-  p.nb = nb;
-  p.chunks = (nblk + nb - 1) / nb;
-  p.tmem_cols = next_pow2((nb + 1) * p.n_pad < 32 ? 32 : (nb + 1) * p.n_pad);
+  int chunks = (kAttnTargetCtas + per_chunk - 1) / per_chunk;
+  chunks = chunks < 1 ? 1 : (chunks > p.nblk ? p.nblk : chunks);
+  p.nb = (p.nblk + chunks - 1) / chunks;
+  p.chunks = (p.nblk + p.nb - 1) / p.nb;
+  // a 3-deep ring of 32 KB stages at 16 query rows, 2-deep at 32, so two CTAs
+  // fit on an SM; TMEM: two score slots and O
+  p.stages = p.n_pad <= 16 ? 3 : 2;
+  p.tmem_cols = next_pow2(3 * p.n_pad < 32 ? 32 : 3 * p.n_pad);
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(tpb::kAttnHeadDim));
   const size_t rows = static_cast<size_t>(groups) * nkv * p.chunks * p.n_pad;
   part_o_bytes = (rows * tpb::kAttnHeadDim * 4 + 255) / 256 * 256;
@@ -799,7 +795,7 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
   if (!aligned16(workspace)) return TP_ERR_ALIGN;
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  const int smem = tpb::attn_smem_bytes(p.nb, p.n_pad);
+  const int smem = tpb::attn_smem_bytes(p.stages, p.n_pad);
   if (smem > dev->max_smem) return TP_ERR_UNSUPPORTED;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + po);
@@ -845,9 +841,10 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = static_cast<unsigned>(nattr);
-    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel, tq, tk, tv, p),
-                 "launch attn_decode_kernel"))
-      return TP_ERR_CUDA;
+    const cudaError_t e = p.n_pad <= 16
+                              ? cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel<16>, tq, tk, tv, p)
+                              : cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel<32>, tq, tk, tv, p);
+    if (!cuda_ok(e, "launch attn_decode_kernel")) return TP_ERR_CUDA;
   }
   // 3. merge the chunks of every (token, query head) in chunk order
   {
