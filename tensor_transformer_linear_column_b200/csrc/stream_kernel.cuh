@@ -51,13 +51,15 @@
 //
 // 8-bit weights (kW8): the weight is FP8 E4M3 with one fp32 scale per row
 // (drpranayjha.com "AI Infrastructure series, Part 5", section "Reason 2":
-// decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 into the
-// upper half of the stage's 16 KB weight tile; the four epilogue warps, idle
-// while the weights stream, rewrite it in place as the bf16 tile the MMA reads
-// (exact: every E4M3 value is a bf16 value), and the row scale multiplies the
-// fp32 sum before bias and activation.
-// The MMAs and everything after them are those of the bf16 kernel; HBM traffic
-// is halved.
+// decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 codes
+// into the stage (64-byte swizzle, so a thread reading its own row's 64 codes
+// hits every bank once per eight lanes); the four epilogue warps, idle while
+// the weights stream, convert them (exact: every E4M3 value is a bf16 value)
+// and store the bf16 tile straight into tensor memory, one row per thread, as
+// the MMA's A operand.  So per k-block shared memory carries only the codes
+// (written by TMA, read once) and x, not a bf16 tile written and read again.
+// Four TMEM A slots decouple conversion from the MMAs.  The row scale
+// multiplies the fp32 sum before bias and activation; HBM traffic is halved.
 //
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
 // push and reduce, and with 8-bit weights first convert the weight tiles;
@@ -98,17 +100,28 @@ constexpr int kStreamTileM = 128;
 constexpr int kStreamTileK = 64;
 constexpr int kStreamW8Bytes = kStreamTileM * kStreamTileK;  // one k-block of 8-bit W: 8 KB
 constexpr int kStreamMaxStages = 8;
+constexpr int kStreamMaxStagesW8 = 12;  // 8 KB code stages: a deeper ring in the same memory
 constexpr int kStreamReleaseBack = 2;  // boxes still to issue when the next grid is released
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
+constexpr int kStreamW8Slots = 4;   // 8-bit weights: bf16 k-blocks in TMEM (A operand slots)
+
+// TMEM columns a CTA allocates: two accumulator regions of tmem_cols each,
+// and with 8-bit weights four 32-column A slots.
+__host__ __device__ inline int stream_tmem_alloc_cols(int tmem_cols, bool w8) {
+  const int need = 2 * tmem_cols + (w8 ? kStreamW8Slots * 32 : 0);
+  int c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
 
 // Shared memory layout (dynamic, base rounded up to 1024 B):
 //   [0, stages * stage_bytes)   pipeline: per stage kpb W tiles (16 KB each) then kpb x
 //                               tiles (t_pad * 128 B each); with 8-bit weights (kpb = 1)
-//                               the 8 KB E4M3 tile [128][64] bytes lands in the upper
-//                               half of the W tile and is converted in place
+//                               the W tile is the 8 KB E4M3 tile [128][64] bytes
+//                               (64-byte swizzle), converted into TMEM
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
-//   conv[stages] (8-bit weights: tile converted), tmem slot, abort flag
+//   a_full[4], a_empty[4] (8-bit weights: TMEM A slots), tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
 //
 // Row stride RS of the receive buffer: T rounded up to 4 floats (one 16-byte
@@ -127,9 +140,16 @@ __host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, in
   return stages * stage_bytes + stream_recv_bytes(T, csize);
 }
 
-__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize) {
+// Barriers after the data: full[stages], empty[stages], seg_full[2],
+// seg_empty[2], final[2], recv, then `stream_extra_bars` more: a_full[4] and
+// a_empty[4] with 8-bit weights, an unused [stages] otherwise.
+__host__ __device__ inline int stream_extra_bars(int stages, bool w8) {
+  return w8 ? 2 * kStreamW8Slots : stages;
+}
+
+__host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize, bool w8) {
   return 1024 /*alignment slack*/ + stream_data_bytes(stages, stage_bytes, T, csize) +
-         (3 * stages + 7) * 8 + 16;
+         (2 * stages + 7 + stream_extra_bars(stages, w8)) * 8 + 16;
 }
 
 // Epilogue of one value: bias, activation, round to bf16, store.
@@ -203,8 +223,10 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   uint64_t* seg_empty = bars + 2 * p.stages + 2;  // [2]
   uint64_t* final_bar = bars + 2 * p.stages + 4;  // [2], one per MMA issuer
   uint64_t* recv_bar = bars + 2 * p.stages + 6;   // bytes of the peers' partials for my rows
-  uint64_t* conv_bar = bars + 2 * p.stages + 7;   // [stages]: 8-bit tile converted to bf16
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv_bar + p.stages);
+  uint64_t* a_full = bars + 2 * p.stages + 7;     // [4]: 8-bit weights, A slot converted (4 warps)
+  uint64_t* a_empty = a_full + kStreamW8Slots;    // [4]: A slot read by the MMAs (commit)
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(bars + 2 * p.stages + 7 + stream_extra_bars(p.stages, kW8));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -223,13 +245,20 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   const int box_seg = nbox / p.spc;  // boxes per accumulation segment
   // two TMEM regions: the two issuers' accumulators (one segment), or
   // alternate shards (several segments)
-  const uint32_t tcols_alloc = static_cast<uint32_t>(2 * p.tmem_cols);
+  // (8-bit weights: then four A slots of 32 columns, one bf16 k-block each)
+  const uint32_t a_col0 = static_cast<uint32_t>(2 * p.tmem_cols);
+  const uint32_t tcols_alloc = static_cast<uint32_t>(stream_tmem_alloc_cols(p.tmem_cols, kW8));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
-      mbar_init(smem_u32(&conv_bar[s]), 4);  // one arrive per converting warp
+    }
+    if constexpr (kW8) {
+      for (int a = 0; a < kStreamW8Slots; ++a) {
+        mbar_init(smem_u32(&a_full[a]), 4);  // one arrive per converting warp
+        mbar_init(smem_u32(&a_empty[a]), 1);
+      }
     }
     for (int b = 0; b < 2; ++b) {
       // one segment: both issuers commit to seg_full[0]
@@ -255,14 +284,11 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   if (multi) cluster_arrive_relaxed();
 
   const uint32_t x_bytes = static_cast<uint32_t>(p.t_pad) * kStreamTileK * 2;
-  const uint32_t w_bytes = kStreamTileM * kStreamTileK * 2;  // one k-block of W: 16 KB
+  // one k-block of W: 16 KB of bf16, or 8 KB of E4M3 codes (kpb == 1)
+  const uint32_t w_bytes = kW8 ? kStreamW8Bytes : kStreamTileM * kStreamTileK * 2;
   const uint32_t xoff = static_cast<uint32_t>(kpb) * w_bytes;  // x tiles follow the W tiles
-  // 8-bit weights (kpb == 1): the 8 KB E4M3 tile lands in the second half of
-  // the stage's bf16 weight tile and is converted in place
-  const uint32_t w8off = w_bytes - kStreamW8Bytes;
-  const uint32_t wdst = kW8 ? w8off : 0u;
-  const uint32_t tx_bytes =
-      kW8 ? kStreamW8Bytes + x_bytes : static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
+  const uint32_t wdst = 0u;
+  const uint32_t tx_bytes = static_cast<uint32_t>(kpb) * (w_bytes + x_bytes);
 
   if (warp == kStreamProducerWarp) {
     if (lane == 0) {
@@ -350,6 +376,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       int i = 0;        // box index
       int s = 0;        // its stage
       uint32_t ph = 0u;  // its pass parity
+      // 8-bit weights: box i's A slot is i % 4, its pass parity (i / 4) % 2
       for (int g = 0; ok && g < p.spc; ++g) {
         const int region = kShards ? (g & 1) : me;
         if (kShards && g >= 2) {
@@ -365,23 +392,38 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         bool first = true;
         for (; i < end; ++i) {
           if (kShards || (s & 1) == me) {
-            if (!wait_parity(smem_u32(kW8 ? &conv_bar[s] : &full_bar[s]), ph, abort_flag)) {
+            const int a = i & (kStreamW8Slots - 1);
+            const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
+            if (!wait_parity(smem_u32(kW8 ? &a_full[a] : &full_bar[s]), kW8 ? aph : ph,
+                             abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t st = static_cast<uint32_t>(s * p.stage_bytes);
             for (int c = 0; c < kpb; ++c) {
-              const uint64_t da = desc0 + ((st + static_cast<uint32_t>(c) * w_bytes) >> 4);
               const uint64_t db = desc0 + ((st + xoff + static_cast<uint32_t>(c) * x_bytes) >> 4);
+              if constexpr (kW8) {
+                // A: the converted bf16 k-block in TMEM slot a, 8 columns per K = 16
+                const uint32_t ta = tmem_d + a_col0 + static_cast<uint32_t>(a * 32);
 #pragma unroll
-              for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
-                umma_bf16(d, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2),
-                          idesc, first ? 0u : 1u);
-                first = false;
+                for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
+                  umma_bf16_ta(d, ta + static_cast<uint32_t>(kk * 8), db + static_cast<uint64_t>(kk * 2),
+                               idesc, first ? 0u : 1u);
+                  first = false;
+                }
+              } else {
+                const uint64_t da = desc0 + ((st + static_cast<uint32_t>(c) * w_bytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
+                  umma_bf16(d, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2),
+                            idesc, first ? 0u : 1u);
+                  first = false;
+                }
               }
             }
             umma_commit(smem_u32(&empty_bar[s]));
+            if constexpr (kW8) umma_commit(smem_u32(&a_empty[a]));
           }
           if (++s == p.stages) {
             s = 0;
@@ -401,49 +443,41 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
     if constexpr (kW8) {
-      // ---------------- warps 0-3, first: E4M3 -> bf16, in place.  A box's
-      // 64-byte E4M3 rows occupy the upper half of the 16 KB tile whose 128-byte
-      // bf16 rows they become, so all 128 threads read their codes into
-      // registers before any thread writes (named barrier 1, reached by every
-      // converter thread once per box whatever its wait returned).  Thread t
-      // takes the 16 codes in chunk c = t % 4 of rows t / 4 + 32 pass: a warp
-      // reads 512 contiguous bytes per pass (no bank conflicts; a
-      // thread-per-row walk at a 64-byte stride puts 16 lanes on the same
-      // banks).  The 16 bf16 values are 16-byte chunks 2c and 2c + 1 of the
-      // row in the 128-byte-swizzled layout of a TMA tile (chunk j of row r at
-      // chunk j ^ (r % 8)), which the MMA descriptor expects.
-      constexpr int kPasses = kStreamTileM / 32;
+      // ---------------- warps 0-3, first: E4M3 -> bf16 into TMEM.  Thread t
+      // owns TMEM lane t = weight row t of the tile: it reads its row's 64
+      // codes (four 16-byte chunks; chunk c sits at chunk c ^ ((t / 2) % 4) of
+      // the row under the 64-byte swizzle), converts them and stores the 64
+      // bf16 values as 32 columns of A slot i % 4.  Every converter thread
+      // takes every box in order, whatever its waits returned, so the warps'
+      // arrivals stay matched.
       const int t = static_cast<int>(threadIdx.x);
-      const int c = t & 3;
+      const uint32_t lane_addr_c = static_cast<uint32_t>(warp * 32) << 16;
+      const int sw = (t >> 1) & 3;
       int s = 0;
       uint32_t ph = 0u;
       bool ok = true;
       for (int i = 0; i < nbox; ++i) {
+        const int a = i & (kStreamW8Slots - 1);
+        const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
         ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
-        uint8_t* st = smem + s * p.stage_bytes;
-        uint4 q[kPasses];
-#pragma unroll
-        for (int pass = 0; pass < kPasses; ++pass) {
-          const int r = pass * 32 + (t >> 2);
-          q[pass] = ok ? *reinterpret_cast<const uint4*>(st + w8off + r * kStreamTileK + c * 16)
-                       : make_uint4(0u, 0u, 0u, 0u);
-        }
-        named_barrier_sync(1, 128);
+        ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
         if (ok) {
+          const uint8_t* row = smem + s * p.stage_bytes + t * kStreamTileK;
+          uint32_t w[32];
 #pragma unroll
-          for (int pass = 0; pass < kPasses; ++pass) {
-            const int r = pass * 32 + (t >> 2);
-            uint8_t* dst = st + r * 128;
-            const int sw = r & 7;
-            *reinterpret_cast<uint4*>(dst + (((2 * c) ^ sw) * 16)) =
-                e4m3x8_to_bf16x8(make_uint2(q[pass].x, q[pass].y));
-            *reinterpret_cast<uint4*>(dst + (((2 * c + 1) ^ sw) * 16)) =
-                e4m3x8_to_bf16x8(make_uint2(q[pass].z, q[pass].w));
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+            const uint4 lo = e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
+            const uint4 hi = e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
+            w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+            w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
           }
-          fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+          tmem_st32(tmem_d + lane_addr_c + a_col0 + static_cast<uint32_t>(a * 32), w);
+          tmem_wait_st();
         }
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&conv_bar[s]));
+        if (lane == 0) mbar_arrive(smem_u32(&a_full[a]));
         if (++s == p.stages) {
           s = 0;
           ph ^= 1u;

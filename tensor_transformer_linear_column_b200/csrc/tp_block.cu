@@ -185,8 +185,9 @@ bool make_tmap_blocks(CUtensorMap* map, const void* base, uint64_t rows, uint64_
   return ok;
 }
 
-// Same view of a row-major [rows, cols] 8-bit matrix, unswizzled: a box
-// {64, box_rows, 1} lands as [box_rows][64] bytes.
+// Same view of a row-major [rows, cols] 8-bit matrix with 64-byte swizzling:
+// a box {64, box_rows, 1} lands as [box_rows][64] bytes, 16-byte chunk c of
+// row r stored at chunk c ^ ((r / 2) % 4).
 bool make_tmap_blocks_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                          uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -196,7 +197,7 @@ bool make_tmap_blocks_u8(CUtensorMap* map, const void* base, uint64_t rows, uint
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   if (!ok) cuda_ok(cudaErrorInvalidValue, "cuTensorMapEncodeTiled (8-bit blocks)");
@@ -263,6 +264,15 @@ StreamGeometry stream_geometry(int N, int kb_total, int shards, int t_pad, int s
   return fallback;
 }
 
+// Shared memory per SM (B200: 228 KB) and the 1 KB the hardware reserves per
+// CTA: the least dynamic shared memory per CTA that lets at most `ctas` CTAs
+// share an SM.
+constexpr int kSmemPerSm = 228 * 1024;
+constexpr int kSmemReservedPerCta = 1024;
+inline int stream_smem_for_ctas(int ctas) {
+  return kSmemPerSm / (ctas + 1) - kSmemReservedPerCta + 1;
+}
+
 // The sizes of a streaming launch (everything but pointers and options):
 // geometry, ring depth, box size, shared memory.  Host arithmetic only; the
 // device enters through max_smem.  TP_ERR_UNSUPPORTED if it does not fit.
@@ -276,7 +286,9 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
   p.kb_total = K / tpb::kStreamTileK;
   p.t_pad = (T + 15) / 16 * 16;
   p.tmem_cols = next_pow2(p.t_pad < 32 ? 32 : p.t_pad);
-  p.stage_bytes = (tpb::kStreamTileM + p.t_pad) * tpb::kStreamTileK * 2;
+  // one k-block of W (16 KB of bf16, or 8 KB of E4M3 codes) and of x
+  p.stage_bytes = (w8 ? tpb::kStreamW8Bytes : tpb::kStreamTileM * tpb::kStreamTileK * 2) +
+                  p.t_pad * tpb::kStreamTileK * 2;
   p.shards = shards;
   p.csize = geo.csize;
   p.jsplit = geo.jsplit;
@@ -295,7 +307,6 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
         static_cast<long>(hi - lo) * tpb::kStreamTileM * tpb::kStreamTileK * (w8 ? 1 : 2);
     const int budget = (w_cta >= 256 * 1024 ? 110 : 72) * 1024 -
                        tpb::stream_recv_bytes(p.T, p.csize);
-    // one k-block of W (bf16) and x; an 8-bit tile is converted in place
     const int kb_bytes = p.stage_bytes;
     bool even = p.spc == 1;
     for (int r = 0; even && r < p.csize; ++r) {
@@ -306,7 +317,8 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
     int kbs = budget / kb_bytes;
     kbs = kbs < 3 ? 3 : kbs;
     int stages = kbs / p.kpb;
-    stages = stages < 2 ? 2 : (stages > tpb::kStreamMaxStages ? tpb::kStreamMaxStages : stages);
+    const int max_stages = w8 ? tpb::kStreamMaxStagesW8 : tpb::kStreamMaxStages;
+    stages = stages < 2 ? 2 : (stages > max_stages ? max_stages : stages);
     p.stages = stages;
     p.stage_bytes = p.kpb * kb_bytes;
     // short streams: two more boxes into L2 before the grid wait (measured
@@ -316,9 +328,19 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
   }
   // large T: the receive buffer leaves room for two stages only
   while (p.stages > 2 &&
-         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize) > max_smem)
+         tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8) > max_smem)
     --p.stages;
-  smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize);
+  smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8);
+  // The CTAs that share an SM must fit their TMEM allocations together: a CTA
+  // whose allocation waited for a cluster peer on the same SM to finish would
+  // wait for ever (the peer waits for it at the cluster barrier).  Shared
+  // memory caps the CTAs per SM, so ask for enough of it.
+  {
+    const int alloc = tpb::stream_tmem_alloc_cols(p.tmem_cols, w8);
+    const int max_ctas = 512 / alloc;
+    const int floor_smem = stream_smem_for_ctas(max_ctas);
+    if (smem < floor_smem) smem = floor_smem;
+  }
   return smem > max_smem ? TP_ERR_UNSUPPORTED : TP_OK;
 }
 

@@ -301,12 +301,13 @@ def test_stream_plan_of_the_sq4096_decode_launches():
 
 
 def test_stream_plan_ring_depths_of_the_70b_decode():
-    # 8-bit tiles are converted in place, so a stage holds one bf16 tile + x
-    for T, stages in ((1, 6), (16, 6), (64, 4)):
+    # 8-bit codes are converted into tensor memory, so a stage holds only the
+    # 8 KB code tile + x: a deeper ring in the same shared memory
+    for T, stages in ((1, 11), (16, 11), (64, 6)):
         p = tp.tp_stream_plan(T, 8192, 28672, 1, w8=True)
         assert p["stages"] == stages and p["kblocks_per_box"] == 1
         t_pad = (T + 15) // 16 * 16
-        assert p["stage_bytes"] == (128 + t_pad) * 64 * 2
+        assert p["stage_bytes"] == (64 + t_pad) * 64 * 2
     # bf16 up-projection at T = 1: two k-blocks per box, three boxes in flight
     p = tp.tp_stream_plan(1, 8192, 28672)
     assert p["kblocks_per_box"] == 2 and p["stages"] == 3
@@ -336,9 +337,18 @@ def test_stream_plan_invariants(w8):
                 else:
                     assert p["jsplit"] == 1 and p["shards_per_cta"] * p["cluster"] == shards
                     assert t_pad <= 64  # the running sum of several shards lives in registers
-                assert 2 <= p["stages"] <= 8
+                assert 2 <= p["stages"] <= (12 if w8 else 8)
                 assert p["kblocks_per_box"] in (1, 2)
-                assert p["stage_bytes"] == p["kblocks_per_box"] * (128 + t_pad) * 128
+                w_row = 64 if w8 else 128  # bytes per weight row of a k-block
+                assert p["stage_bytes"] == p["kblocks_per_box"] * (w_row + t_pad) * 128
+                # the CTAs an SM can hold never need more TMEM than it has:
+                # two accumulator regions (+ four 32-column A slots for 8-bit)
+                tcols = max(32, 1 << (t_pad - 1).bit_length())
+                need = 2 * tcols + (128 if w8 else 0)
+                alloc = 1 << (need - 1).bit_length()
+                by_regs = 2 if p["shards_per_cta"] > 1 else 3
+                by_smem = (228 * 1024) // (p["smem_bytes"] + 1024)
+                assert min(by_regs, by_smem) * alloc <= 512, (T, K, N, shards, w8, p)
                 assert p["smem_bytes"] <= max_smem
                 assert p["smem_bytes"] >= p["stages"] * p["stage_bytes"]
                 if w8:
