@@ -131,3 +131,32 @@ def test_attn_decode_chained_steps_match_one_prefill():
     cache = [(kc[s * kh:(s + 1) * kh, :1200], vc[s * kh:(s + 1) * kh, :1200]) for s in range(t)]
     ref, _ = oracle.attn_core(qkv, nq, nkv, D, t, cache)
     _parity(torch.cat(outs, 0), ref, "three chained steps")
+
+
+def test_attn_decode_bench_workload_sizes():
+    # the bench workload itself: 64K cached tokens of the 70B head layout,
+    # T = 1, 2, 4, in the launch configuration bench.py times (programmatic
+    # dependent launch with static-weight prefetch), against the oracle
+    dev = _dev()
+    cfg = workloads.CONFIGS["attn70b_decode"]
+    nq, nkv, t = cfg.n_q_heads, cfg.n_kv_heads, cfg.tp_degrees[0]
+    k, v = workloads.attn_decode_cache(cfg)
+    kh = nkv // t
+    cache = [(k[s * kh:(s + 1) * kh], v[s * kh:(s + 1) * kh]) for s in range(t)]
+    max_len = cfg.past + max(cfg.tokens)
+    kd = torch.empty((nkv, max_len, D), dtype=torch.bfloat16, device=dev)
+    vd = torch.empty_like(kd)
+    prev = tp.tp_get_launch_options()
+    tp.tp_set_launch_options(tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS)
+    try:
+        for T in cfg.tokens:
+            kd[:, :cfg.past].copy_(k)
+            vd[:, :cfg.past].copy_(v)
+            qkv = workloads.attn_decode_qkv(cfg, T)
+            ref, _ = oracle.attn_core(qkv, nq, nkv, D, t, cache)
+            ctx = tp.tp_attn_decode(qkv.to(dev), kd, vd, cfg.past, nq, nkv, D, t)
+            torch.cuda.synchronize()
+            _parity(ctx, ref, f"bench workload T={T}")
+    finally:
+        tp.tp_set_launch_options(prev)
+    assert tp.tp_device_error_check() == tp.TP_OK

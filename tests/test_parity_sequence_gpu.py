@@ -61,3 +61,27 @@ def test_sp_region_bit_identical_on_repeat():
     b = tp.tp_sp_add_rmsnorm(y, res, g, 8)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_sp405b_bench_workload_sampled_rows():
+    # the bench workload (T = 8192 token rows of H = 16384, t = 8) in the
+    # bench's launch configuration; the oracle checks 64 seeded rows
+    dev = _dev()
+    cfg = workloads.CONFIGS["sp405b"]
+    T = cfg.tokens[0]
+    d = workloads.sp_norm_inputs(cfg, T)
+    rows = workloads.sample_rows(T, 64)
+    r_ref, n_ref = oracle.sp_residual_norm([oracle.to_f64(d["y"][rows])], None,
+                                           d["residual"][rows], d["gamma"], 1)
+    prev = tp.tp_get_launch_options()
+    tp.tp_set_launch_options(tp.TP_OPT_PDL | tp.TP_OPT_STATIC_WEIGHTS)
+    try:
+        r, n = tp.tp_sp_add_rmsnorm(d["y"].to(dev), d["residual"].to(dev), d["gamma"].to(dev),
+                                    cfg.tp_degrees[0])
+        torch.cuda.synchronize()
+    finally:
+        tp.tp_set_launch_options(prev)
+    idx = torch.tensor(rows, device=dev)
+    _parity(r[idx], r_ref, "sp405b r")
+    _parity(n[idx], n_ref, "sp405b n")
+    assert tp.tp_device_error_check() == tp.TP_OK
