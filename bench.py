@@ -61,6 +61,7 @@ LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # default (timed steps, warm-up steps) per workload: about a second of timed work
 DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "attn70b_decode": (5000, 50),
+                 "mlp70b_bwd": (100, 5),
                  "sp405b": (2000, 20),
                  "mlp70b": (2000, 50),
                  "mlp70b_w8": (2000, 50), "sq4096": (20000, 200), "tiny": (20000, 200)}
@@ -271,6 +272,23 @@ class Workload:
             self.ws = torch.empty(max(tp.tp_attn_decode_workspace_bytes(
                 T, cfg.past, cfg.n_q_heads, cfg.n_kv_heads, d) for T in self.Ts),
                 dtype=torch.uint8, device=device)
+        elif name == "mlp70b_bwd":
+            self.t = tp_degree or cfg.tp_degrees[-1]
+            self.Ts = list(tokens or cfg.tokens)
+            d = workloads.mlp_inputs(cfg, self.Ts[0])
+            self.xs = {T: workloads.mlp_x(cfg, T) for T in self.Ts}
+            self.dy = {T: workloads.mlp_dy(cfg, T).to(device) for T in self.Ts}
+            self.weight_bytes = (d["w1"].numel() + d["w2"].numel()) * 2
+            self.hidden_in = self.hidden_out = cfg.hidden
+            self.weights = [(d["w1"].to(device), d["w2"].to(device))]
+            F, H = cfg.ffn, cfg.hidden
+            self.grads = {T: {"dw1": torch.empty((F, H), dtype=torch.bfloat16, device=device),
+                              "dw2": torch.empty((H, F), dtype=torch.bfloat16, device=device),
+                              "db1": torch.empty((F,), dtype=torch.bfloat16, device=device),
+                              "db2": torch.empty((H,), dtype=torch.bfloat16, device=device)}
+                          for T in self.Ts}
+            self.ws = torch.empty(max(tp.tp_mlp_backward_workspace_bytes(T, F) for T in self.Ts),
+                                  dtype=torch.uint8, device=device)
         elif name == "sp405b":
             self.t = tp_degree or cfg.tp_degrees[0]
             self.Ts = list(tokens or cfg.tokens)
@@ -300,7 +318,7 @@ class Workload:
                     self.weights.append(base.clone())
         self.tokens_per_step = sum(self.Ts)
         self.launches_per_step = len(self.Ts) * {"sq4096": 1, "attn70b_decode": 3,
-                                                 "sp405b": 1}.get(name, 2)
+                                                 "sp405b": 1, "mlp70b_bwd": 7}.get(name, 2)
 
     def step(self, i: int, xs=None, outs=None):
         tp = self.tp
@@ -315,6 +333,16 @@ class Workload:
             elif self.name == "mlp70b_w8":
                 tp.tp_mlp_forward_w8(xs[T], w[0], w[1], None, w[2], w[3], None, self.t,
                                      self.cfg.act, out=outs[T], workspace=self.ws)
+            elif self.name == "mlp70b_bwd":
+                gr = self.grads[T]
+                st = tp.load().tp_mlp_backward(
+                    xs[T].data_ptr(), w[0].data_ptr(), None, w[1].data_ptr(),
+                    self.dy[T].data_ptr(), T, self.cfg.hidden, self.cfg.ffn, self.t,
+                    tp.ACTS[self.cfg.act], outs[T].data_ptr(), gr["dw1"].data_ptr(),
+                    gr["db1"].data_ptr(), gr["dw2"].data_ptr(), gr["db2"].data_ptr(),
+                    self.ws.data_ptr(), self.ws.numel(), torch.cuda.current_stream().cuda_stream)
+                if st != tp.TP_OK:
+                    raise tp.TPError(st, "tp_mlp_backward")
             elif self.name == "sp405b":
                 tp.tp_sp_add_rmsnorm(xs[T], self.res[T], w, self.t, 1e-5, r_out=self.r_out[T],
                                      n_out=outs[T])
@@ -346,11 +374,12 @@ class Workload:
         return b
 
     def step_flops(self):
-        """2 T per weight element (bf16 weights: 2 bytes per element)."""
+        """2 T per weight element (bf16 weights: 2 bytes per element); the
+        backward pass makes five GEMMs of the layer's size per step."""
         f = 0
         for T in self.Ts:
             f += 2 * T * self.weight_bytes // 2
-        return f
+        return f * 5 // 2 if self.name == "mlp70b_bwd" else f
 
     def bound(self):
         if self.name == "sp405b":
@@ -376,7 +405,15 @@ class _OracleRunner:
         cfg = workloads.CONFIGS[name]
         self.name = name
         self.cfg = cfg
-        if name == "sp405b":
+        if name == "mlp70b_bwd":
+            self.t = t or cfg.tp_degrees[-1]
+            T0 = cfg.tokens[0]
+            d = workloads.mlp_inputs(cfg, T0)
+            rows = workloads.sample_rows(T0, cfg.sample_rows)
+            self.x, self.dy = d["x"][rows], workloads.mlp_dy(cfg, T0)[rows]
+            self.w1, self.w2 = d["w1"], d["w2"]
+            self.n_out = cfg.hidden
+        elif name == "sp405b":
             self.t = t or cfg.tp_degrees[0]
             T0 = cfg.tokens[0]
             d = workloads.sp_norm_inputs(cfg, T0)
@@ -424,11 +461,18 @@ class _OracleRunner:
             return self.x.shape[0]
         if self.name == "sp405b":
             return self.y.shape[0]
+        if self.name == "mlp70b_bwd":
+            return self.x.shape[0]
         return sum(x.shape[0] for x in self.xs.values())
 
     def run(self, fraction, offset):
         """Compute the step on output-feature block [offset, offset + fraction * n_out)."""
         import oracle
+        if self.name == "mlp70b_bwd":
+            # the backward pass of 64 seeded tokens (weight gradients over them)
+            oracle.mlp_block_backward(self.x, self.w1, None, self.w2, self.dy, self.t,
+                                      self.cfg.act)
+            return 1.0
         if self.name == "sp405b":
             # 64 seeded token rows (rows are independent); one token shard
             oracle.sp_residual_norm([oracle.to_f64(self.y)], None, self.res, self.gamma, 1)
@@ -567,6 +611,8 @@ def workload_config(name, t, options, tokens=None):
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
         "attn70b_decode": "attention core decode, 64 query / 8 key-value heads of 128 (t=8), "
                           "65536 cached tokens, T=1,2,4 new tokens per call",
+        "mlp70b_bwd": "backward pass of the Llama-3-70B-shaped MLP block H=8192 F=28672, GeLU, "
+                      "t=8, T=4096 tokens: dx (fused backward shard sum), dW1, dW2, db1, db2",
         "sp405b": "sequence-parallel region of the 405B-shaped block: residual add + RMSNorm "
                   "of T=8192 token rows of H=16384 in 8 token shards",
         "mlp405b": "405B-shaped MLP prefill H=16384 F=53248, GeLU, T=8192, column-parallel "
@@ -735,7 +781,11 @@ def kernel_durations(wl, stream, reps=5):
     tp = wl.tp
     T = wl.Ts[0]
     out = {}
-    if wl.name == "attn70b":
+    if wl.name == "mlp70b_bwd":
+        # one backward pass: z recompute, dz and h, dx with the shard sum, dW1,
+        # dW2 (five CTA-pair GEMMs) and the two column sums, as one call
+        calls = {"pair_gemm_kernel<backward>:five_gemms": (lambda: wl.step(0), wl.step_flops())}
+    elif wl.name == "attn70b":
         cfg = wl.cfg
         wq, wo = wl.weights[0]
         nctx = cfg.n_q_heads * cfg.head_dim

@@ -164,6 +164,10 @@ CONFIGS: Dict[str, object] = {
     # Llama-3-70B-shaped MLP decode
     "mlp70b": MLPConfig("mlp70b", hidden=8192, ffn=28672, tokens=(1, 16, 64),
                         tp_degrees=(4, 8), act="gelu_tanh", w_std=0.02, b_std=None),
+    # the backward pass of the 70B-shaped MLP over a 4096-token batch (training)
+    "mlp70b_bwd": MLPConfig("mlp70b_bwd", hidden=8192, ffn=28672, tokens=(4096,),
+                            tp_degrees=(8,), act="gelu_tanh", w_std=0.02, b_std=None,
+                            sample_rows=64),
     # the same MLP with 8-bit (E4M3, per-row scale) weights, decode
     "mlp70b_w8": MLPConfig("mlp70b_w8", hidden=8192, ffn=28672, tokens=(1, 16, 64),
                            tp_degrees=(4, 8), act="gelu_tanh", w_std=0.02, b_std=None,
@@ -261,6 +265,11 @@ def sp_norm_inputs(cfg: SPNormConfig, T: int, seed: int = 0) -> Dict[str, torch.
     res = normal_bf16((T, cfg.hidden), 1.0, seed, 800 + int(T))
     gamma = (1.0 + normal_bf16((cfg.hidden,), 0.1, seed, 701).float()).to(torch.bfloat16)
     return {"y": y, "residual": res, "gamma": gamma}
+
+
+def mlp_dy(cfg: MLPConfig, T: int, seed: int = 0) -> torch.Tensor:
+    """The upstream gradient dy [T, H] of the block's output, N(0, 1) bf16."""
+    return normal_bf16((T, cfg.hidden), 1.0, seed, 900 + int(T))
 
 
 def quantize_e4m3_rows(w: torch.Tensor, rows_per_chunk: int = 2048
