@@ -645,6 +645,8 @@ def run_ours(args, world, rank, local):
     init_dist(world, "nccl")
     tp.load()
     tp.tp_set_launch_options(LAUNCH_OPTIONS[args.options])
+    if args.decode_max_tokens is not None:
+        tp.tp_set_decode_max_tokens(args.decode_max_tokens)
     wl = Workload(args.workload, args.tp, dev, rotate=True, tokens=args.tokens)
     stream = torch.cuda.Stream(device=dev)
     K, W = args.steps, args.warmup
@@ -732,7 +734,8 @@ def run_ours(args, world, rank, local):
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0, sigma) bf16 inputs of the workload's shapes)",
-            "config": workload_config(args.workload, wl.t, args.options, args.tokens),
+            "config": dict(workload_config(args.workload, wl.t, args.options, args.tokens),
+                           decode_max_tokens=tp.tp_get_decode_max_tokens()),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": wl.launches_per_step * K,
             "clocks": clocks,
@@ -879,6 +882,9 @@ def parse(argv=None):
     ap.add_argument("--tokens", type=int, nargs="+", default=None,
                     help="override the workload's token counts (smaller captures for ncu); "
                          "not a headline configuration")
+    ap.add_argument("--decode-max-tokens", type=int, default=None,
+                    help="token count up to which calls take the weight-streaming kernel "
+                         "(the library's default is 64)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -28,15 +28,19 @@
 //                              one of two TMEM score slots
 //   softmax of block b         the four epilogue warps (one key per thread):
 //                              mask, the block maximum per query row, the
-//                              running maximum m, p = 2^(s - m) rounded to bf16
-//                              into one of two shared-memory P slots (the next
-//                              MMA's K-major B operand), the running sum l
-//                              rescaled by alpha = 2^(m_old - m), and the
-//                              accumulator O rescaled by alpha in TMEM
-//   O^T[d, n] += V_b^T P_b^T   tcgen05.mma, d as M: V is read MN-major straight
-//                              from its [key][d] tile, keys as K
-// The scores of block b + 1 are computed while block b's softmax runs, and
-// block b's P V product while block b + 1's scores are read.  HBM traffic is
+//                              running maximum m of accumulator b % 2,
+//                              p = 2^(s - m) rounded to bf16 into one of two
+//                              shared-memory P slots (the next MMA's K-major B
+//                              operand), the running sum l rescaled by
+//                              alpha = 2^(m_old - m), and that accumulator
+//                              rescaled by alpha in TMEM
+//   O_{b%2}^T[d, n] += V_b^T P_b^T   tcgen05.mma, d as M: V is read MN-major
+//                              straight from its [key][d] tile, keys as K
+// Even and odd blocks accumulate into separate O's with their own running
+// maxima and sums, merged at the end: block b's softmax then waits only for
+// block b - 2's P V product (long done), never for block b - 1's, so the
+// MMA of one block overlaps the softmax of the next.  The scores of block
+// b + 1 are also computed while block b's softmax runs.  HBM traffic is
 // the cache read once per token group (K and V, 512 bytes per key at d = 128)
 // plus partials of (d + 2) * 4 bytes per query row per chunk.
 #pragma once
@@ -72,10 +76,11 @@ struct AttnParams {
 
 // Shared memory (dynamic, base rounded up to 1024 B): ring [stages][32 KB],
 // Q [2 d halves][n_pad][64] bf16, P [2 slots][2 key halves][n_pad][64] bf16,
-// reduction scratch [2][4][32] floats, m / l / alpha [32] floats, barriers.
+// reduction scratch [2][4][32] floats, m / l [2 accumulators][32] and alpha
+// [32] floats, barriers.
 __host__ __device__ inline int attn_q_bytes(int n_pad) { return n_pad * kAttnHeadDim * 2; }
 __host__ __device__ inline int attn_smem_bytes(int stages, int n_pad) {
-  return 1024 + stages * kAttnBlockBytes + 3 * attn_q_bytes(n_pad) + 2 * 4 * 32 * 4 + 3 * 32 * 4 +
+  return 1024 + stages * kAttnBlockBytes + 3 * attn_q_bytes(n_pad) + 2 * 4 * 32 * 4 + 5 * 32 * 4 +
          (2 * kAttnMaxStages + 10) * 8 + 16;
 }
 
@@ -121,9 +126,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint8_t* ps = qs + 2 * kQHalf;                          // [2 slots][2 halves][kRows][128 B]
   float* red_m = reinterpret_cast<float*>(ps + 4 * kQHalf);  // [4][32]
   float* red_s = red_m + 4 * 32;                             // [4][32]
-  float* m_s = red_s + 4 * 32;                               // [32] running maximum
-  float* l_s = m_s + 32;                                     // [32] running sum
-  float* a_s = l_s + 32;                                     // [32] this block's alpha
+  float* m_s = red_s + 4 * 32;                               // [2][32] running maxima
+  float* l_s = m_s + 2 * 32;                                 // [2][32] running sums
+  float* a_s = l_s + 2 * 32;                                 // [32] this block's alpha
   uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + 32);
   uint64_t* full_bar = bars;                         // [kAttnMaxStages]
   uint64_t* empty_bar = bars + kAttnMaxStages;       // [kAttnMaxStages]
@@ -131,7 +136,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* s_full = q_bar + 1;                      // [2] scores of a block in TMEM slot
   uint64_t* s_free = q_bar + 3;                      // [2] slot read by the softmax (128)
   uint64_t* p_full = q_bar + 5;                      // [2] P slot written, O rescaled (128)
-  uint64_t* o_done = q_bar + 7;                      // [2] the P V product of the slot done
+  uint64_t* o_done = q_bar + 7;                      // [2] the P V product into O_slot done
   uint64_t* final_bar = q_bar + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -171,7 +176,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S slots at columns 0 and kRows, O at 2 kRows
+  // S slots at columns 0 and kRows, O_0 at 2 kRows, O_1 at 3 kRows
+  const uint32_t tmem = *tmem_slot;
   const uint32_t o_col = 2u * kRows;
 
   // load / MMA item i: K_0, then K_b, V_{b-1} for b = 1 .. nbc-1, then V_{nbc-1}
@@ -273,10 +279,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
           for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk) {
             const uint32_t hk = static_cast<uint32_t>(kk >> 2), ck = static_cast<uint32_t>(kk & 3);
-            umma_bf16(tmem + o_col,
+            umma_bf16(tmem + o_col + static_cast<uint32_t>(slot * kRows),
                       desc_mnmajor_sw128(st + static_cast<uint32_t>(kk) * 2048u, kAttnHalfBytes),
                       desc_kmajor_sw128(pb + hk * kQHalf + ck * 32u), idesc_o,
-                      (b > 0 || kk > 0) ? 1u : 0u);
+                      (b >= 2 || kk > 0) ? 1u : 0u);
           }
           umma_commit(smem_u32(&empty_bar[s]));
           umma_commit(smem_u32(&o_done[slot]));
@@ -309,8 +315,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       lim[j] = tok < p.T ? p.past + tok : -1;
     }
     if (et < kRows) {
-      m_s[et] = neg_inf();
-      l_s[et] = 0.0f;
+      m_s[et] = m_s[32 + et] = neg_inf();
+      l_s[et] = l_s[32 + et] = 0.0f;
     }
     // P half (key / 64) of row n: 128-byte rows, 16-byte chunk (key % 64) / 8
     // stored at chunk ^ (n % 8)
@@ -348,22 +354,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (lane == 0) red_m[q4 * 32 + j] = mx;
       }
       named_barrier_sync(1, 128);
+      float* ms = m_s + slot * 32;  // accumulator b % 2's running state
+      float* ls = l_s + slot * 32;
       if (et < kRows) {
         const float mb = fmaxf(fmaxf(red_m[et], red_m[32 + et]), fmaxf(red_m[64 + et], red_m[96 + et]));
-        const float mo = m_s[et];
+        const float mo = ms[et];
         const float mn = fmaxf(mo, mb);
         a_s[et] = mo == neg_inf() ? 0.0f : exp2f(mo - mn);
-        m_s[et] = mn;
+        ms[et] = mn;
       }
       named_barrier_sync(1, 128);
-      // the P slot is free once the P V product of block b - 2 is done
+      // the P slot and accumulator b % 2 are free once block b - 2's P V
+      // product is done
       if (b >= 2)
         ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[slot]),
                                                        ((b - 2) >> 1) & 1, abort_flag));
       uint8_t* pslot = ps + static_cast<size_t>(slot) * 2u * kQHalf + static_cast<size_t>(r >> 6) * kQHalf;
 #pragma unroll
       for (int j = 0; j < kRows; ++j) {
-        const float m = m_s[j];
+        const float m = ms[j];
         const float e = sc[j] == neg_inf() ? 0.0f : exp2f(sc[j] - m);
         const __nv_bfloat16 hb = __float2bfloat16_rn(e);
         *reinterpret_cast<__nv_bfloat16*>(pslot + j * 128 + ((kc ^ (j & 7)) << 4) + kw) = hb;
@@ -374,55 +383,75 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       named_barrier_sync(1, 128);
       if (et < kRows)
-        l_s[et] = fmaf(l_s[et], a_s[et],
-                       ((red_s[et] + red_s[32 + et]) + red_s[64 + et]) + red_s[96 + et]);
-      // O (the P V products of blocks < b) times alpha, once block b - 1's is done
-      if (b >= 1) {
-        ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[(b - 1) & 1]),
-                                                       ((b - 1) >> 1) & 1, abort_flag));
+        ls[et] = fmaf(ls[et], a_s[et],
+                      ((red_s[et] + red_s[32 + et]) + red_s[64 + et]) + red_s[96 + et]);
+      // O_{b%2} (the P V products of blocks b - 2, b - 4, ...) times alpha;
+      // block b - 2's product was waited for above
+      if (b >= 2 && ok) {
         tc_fence_after();
-        if (ok) {
-          uint32_t o[kRows];
+        const uint32_t oc = o_col + static_cast<uint32_t>(slot * kRows);
+        uint32_t o[kRows];
 #pragma unroll
-          for (int c = 0; c < kRows; c += 16)
-            tmem_ld16(tmem + lane_addr + o_col + static_cast<uint32_t>(c),
-                      *reinterpret_cast<uint32_t(*)[16]>(o + c));
-          tmem_wait_ld();
+        for (int c = 0; c < kRows; c += 16)
+          tmem_ld16(tmem + lane_addr + oc + static_cast<uint32_t>(c),
+                    *reinterpret_cast<uint32_t(*)[16]>(o + c));
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < kRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a_s[j]);
+        for (int j = 0; j < kRows; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a_s[j]);
 #pragma unroll
-          for (int c = 0; c < kRows; c += 16)
-            tmem_st16(tmem + lane_addr + o_col + static_cast<uint32_t>(c),
-                      *reinterpret_cast<uint32_t(*)[16]>(o + c));
-          tmem_wait_st();
-        }
+        for (int c = 0; c < kRows; c += 16)
+          tmem_st16(tmem + lane_addr + oc + static_cast<uint32_t>(c),
+                    *reinterpret_cast<uint32_t(*)[16]>(o + c));
+        tmem_wait_st();
       }
       fence_proxy_async_smem();  // P is read by the MMA through the async proxy
       tc_fence_before();
       mbar_arrive(smem_u32(&p_full[slot]));
     }
-    // the last P V product, then the partial: O^T (lane = d, column = query row)
+    // the last P V products of both accumulators, then the partial: the two
+    // merged with weights 2^(m_x - M), M = max(m_0, m_1); O^T has lane = d,
+    // column = query row
     if (nbc > 0)
       ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[(nbc - 1) & 1]),
                                                      ((nbc - 1) >> 1) & 1, abort_flag));
+    if (nbc > 1)
+      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[nbc & 1]),
+                                                     ((nbc - 2) >> 1) & 1, abort_flag));
+    named_barrier_sync(1, 128);  // every thread's m / l updates are visible
+    float* w0s = red_m;          // [32] weight of O_0, [32 + n] weight of O_1
+    if (et < kRows) {
+      const float m0 = m_s[et], m1 = nbc > 1 ? m_s[32 + et] : neg_inf();
+      const float M = fmaxf(m0, m1);
+      const float w0 = m0 == neg_inf() ? 0.0f : exp2f(m0 - M);
+      const float w1 = m1 == neg_inf() ? 0.0f : exp2f(m1 - M);
+      w0s[et] = w0;
+      w0s[32 + et] = w1;
+      const float L = w0 * l_s[et] + (nbc > 1 ? w1 * l_s[32 + et] : 0.0f);
+      const size_t slot = (static_cast<size_t>(grp) * p.nkv + g) * p.chunks + chunk;
+      float* pml = p.part_ml + slot * static_cast<size_t>(kRows) * 2;
+      pml[2 * et] = ok ? M : neg_inf();
+      pml[2 * et + 1] = ok ? L : 0.0f;
+    }
+    named_barrier_sync(1, 128);
     tc_fence_after();
     const size_t slot = (static_cast<size_t>(grp) * p.nkv + g) * p.chunks + chunk;
     float* po = p.part_o + slot * static_cast<size_t>(kRows) * kAttnHeadDim;
 #pragma unroll
     for (int c = 0; c < kRows; c += 16) {
-      uint32_t v[16];
+      uint32_t v0[16], v1[16];
       if (ok) {
-        tmem_ld16(tmem + lane_addr + o_col + static_cast<uint32_t>(c), v);
+        tmem_ld16(tmem + lane_addr + o_col + static_cast<uint32_t>(c), v0);
+        if (nbc > 1) tmem_ld16(tmem + lane_addr + o_col + kRows + static_cast<uint32_t>(c), v1);
         tmem_wait_ld();
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        po[static_cast<size_t>(c + j) * kAttnHeadDim + r] = ok ? __uint_as_float(v[j]) : 0.0f;
-    }
-    if (et < kRows) {
-      float* pml = p.part_ml + slot * static_cast<size_t>(kRows) * 2;
-      pml[2 * et] = ok ? m_s[et] : neg_inf();
-      pml[2 * et + 1] = ok ? l_s[et] : 0.0f;
+      for (int j = 0; j < 16; ++j) {
+        // O_1 is read only when it was written (nbc > 1): unwritten TMEM may
+        // hold any bit pattern, and 0 * NaN is NaN
+        float o = ok ? w0s[c + j] * __uint_as_float(v0[j]) : 0.0f;
+        if (ok && nbc > 1) o = fmaf(w0s[32 + c + j], __uint_as_float(v1[j]), o);
+        po[static_cast<size_t>(c + j) * kAttnHeadDim + r] = o;
+      }
     }
     tc_fence_before();
   }
