@@ -729,13 +729,15 @@ def run_ours(args, world, rank, local):
                          f"(fp64 numpy, {args.workload})"}
 
     if rank == 0:
+        config = workload_config(args.workload, wl.t, args.options, args.tokens)
+        if args.decode_max_tokens is not None:
+            config["decode_max_tokens"] = args.decode_max_tokens
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0, sigma) bf16 inputs of the workload's shapes)",
-            "config": dict(workload_config(args.workload, wl.t, args.options, args.tokens),
-                           decode_max_tokens=tp.tp_get_decode_max_tokens()),
+            "config": config,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": wl.launches_per_step * K,
             "clocks": clocks,
