@@ -36,8 +36,8 @@
 // in a fixed order from its own shared memory, adds the bias, applies the
 // activation and stores bf16.  A split cluster barrier closes the exchange:
 // every thread arrives once it has issued its last remote store, and a CTA
-// waits for that phase before it reads its receive buffer and before it exits,
-// so no CTA leaves while a peer may still write into its shared memory, also
+// waits for that phase before it exits (the owner warps after their sum), so
+// no CTA leaves while a peer may still write into its shared memory, also
 // when a bounded wait has run out somewhere in the cluster (every wait before a
 // send is bounded, so the phase always completes).  Nothing intermediate goes
 // to global memory and there are no atomics, so the result is bit-identical
@@ -618,14 +618,18 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     tmem_dealloc(tmem_d, tcols_alloc);
   }
   if (!multi) return;
-  // no CTA of the cluster exits, and no owner reads its receive buffer, before
-  // every peer has issued all of its remote stores
-  cluster_wait_acquire();
-  if (warp >= 4) return;
+  if (warp >= 4) {
+    // no CTA of the cluster exits before every peer has issued all of its
+    // remote stores (the owner warps take the same wait after their sum)
+    cluster_wait_acquire();
+    return;
+  }
 
   // ---------------- owner: fixed-order sum of the csize partials of its rows.
-  // Every peer always sends its T values per row and has issued them by now,
-  // so this completes within microseconds.
+  // Every peer always sends its T values per row, so this completes within
+  // microseconds; if it ever ran out, the sum would read a partial buffer
+  // (the error word says so) and the closing barrier below still keeps this
+  // CTA alive until every late store has been issued.
   if (!drain_wait(smem_u32(recv_bar), 0, 50ull * 1000ull * 1000ull))
     atomicOr(&g_tp_device_error, kErrTimeout);
   const int RS = stream_recv_stride(p.T);
@@ -669,6 +673,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         if (tok0 + q < p.T) stream_store(p, tok0 + q, n, kW8 ? o[q] * scale_own : o[q], bias_own);
     }
   }
+  cluster_wait_acquire();  // phase 2, see above
 }
 
 }  // namespace tpb
