@@ -453,32 +453,19 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       const int t = static_cast<int>(threadIdx.x);
       const uint32_t lane_addr_c = static_cast<uint32_t>(warp * 32) << 16;
       const int sw = (t >> 1) & 3;
-      // A box's store into TMEM completes while the next box is converted: the
-      // wait for the store and the arrival on a_full come one box later, or at
-      // once when the next box's codes have not landed yet (so the MMAs never
-      // wait on a box that is already converted)
-      int pending = -1;  // box whose tcgen05.st is outstanding
-      auto finish = [&](int box) {
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&a_full[box & (kStreamW8Slots - 1)]));
-      };
       int s = 0;
       uint32_t ph = 0u;
       bool ok = true;
       for (int i = 0; i < nbox; ++i) {
         const int a = i & (kStreamW8Slots - 1);
         const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
-        if (pending >= 0 && !__all_sync(0xffffffffu, mbar_try_wait(smem_u32(&full_bar[s]), ph))) {
-          finish(pending);
-          pending = -1;
-        }
         ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
         ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
-        uint32_t w[32];
-        if (ok) {
+        // the warp stores only when all its lanes' waits succeeded (the store
+        // is warp-wide); every warp arrives for every box whatever happened
+        if (__all_sync(0xffffffffu, ok)) {
           const uint8_t* row = smem + s * p.stage_bytes + t * kStreamTileK;
+          uint32_t w[32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint4 q = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
@@ -487,19 +474,17 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
             w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
             w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
           }
-        }
-        if (pending >= 0) finish(pending);
-        // the warps of a CTA agree on nothing here, so every warp stores and
-        // arrives for every box whatever its waits returned
-        if (__all_sync(0xffffffffu, ok))
           tmem_st32(tmem_d + lane_addr_c + a_col0 + static_cast<uint32_t>(a * 32), w);
-        pending = i;
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&a_full[a]));
         if (++s == p.stages) {
           s = 0;
           ph ^= 1u;
         }
       }
-      if (pending >= 0) finish(pending);
     }
     // ---------------- warps 0-3: drain TMEM, fold shards in order, send rows to their owners
     grid_dependency_wait();
