@@ -51,8 +51,10 @@ namespace tpb {
 
 constexpr int kAttnHeadDim = 128;
 constexpr int kAttnBlockKeys = 128;
-constexpr int kAttnMaxStages = 3;
-constexpr int kAttnThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue
+constexpr int kAttnMaxStages = 2;  // the two MMA issuers rely on exactly two (see below)
+// warp 0 TMA; warp 1 issues the score MMAs, warp 6 the P V MMAs; warps 2-5
+// softmax / epilogue
+constexpr int kAttnThreads = 224;
 constexpr int kAttnBlockBytes = kAttnBlockKeys * kAttnHeadDim * 2;  // 32 KB
 constexpr int kAttnHalfBytes = kAttnBlockBytes / 2;                // one 64-wide d half
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -81,7 +83,7 @@ struct AttnParams {
 __host__ __device__ inline int attn_q_bytes(int n_pad) { return n_pad * kAttnHeadDim * 2; }
 __host__ __device__ inline int attn_smem_bytes(int stages, int n_pad) {
   return 1024 + stages * kAttnBlockBytes + 3 * attn_q_bytes(n_pad) + 2 * 4 * 32 * 4 + 5 * 32 * 4 +
-         (2 * kAttnMaxStages + 10) * 8 + 16;
+         (2 * kAttnMaxStages + 11) * 8 + 16;
 }
 
 // Copy the new tokens' keys and values into the cache: for token i and
@@ -137,8 +139,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* s_free = q_bar + 3;                      // [2] slot read by the softmax (128)
   uint64_t* p_full = q_bar + 5;                      // [2] P slot written, O rescaled (128)
   uint64_t* o_done = q_bar + 7;                      // [2] the P V product into O_slot done
-  uint64_t* final_bar = q_bar + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+  uint64_t* final_bar = q_bar + 9;                   // [2] one per MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -165,7 +167,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(smem_u32(&p_full[i]), 128);
       mbar_init(smem_u32(&o_done[i]), 1);
     }
-    mbar_init(smem_u32(final_bar), 1);
+    mbar_init(smem_u32(&final_bar[0]), 1);
+    mbar_init(smem_u32(&final_bar[1]), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -228,12 +231,21 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 6) {
     if (lane == 0) {
-      // ---------------- MMA issuer, same item order as the loads
+      // ---------------- MMA issuers: warp 1 takes the K items (scores), warp 6
+      // the V items (P V); both walk the load order to track ring stages.
+      // With two stages, stage 0 holds K_0 and then only V blocks, and stage 1
+      // only K blocks except the last item, V_{nbc-1}.  Where a stage changes
+      // hands (K_0 -> V_0, K_{nbc-1} -> V_{nbc-1}), the P V issuer waits for
+      // that block's P first, which needs the block's scores, so the previous
+      // fill has landed: a parity wait never matches an older phase.  The
+      // score MMAs so never queue behind a P V product that waits for its
+      // softmax.
+      const bool pv_role = warp == 6;
       const uint32_t idesc_s = idesc_bf16_f32(128, kRows);               // K, Q both K-major
       const uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, false);  // V^T MN-major, P K-major
-      bool ok = wait_parity(smem_u32(q_bar), 0, abort_flag);
+      bool ok = pv_role || wait_parity(smem_u32(q_bar), 0, abort_flag);
       tc_fence_after();
       int s = 0;
       uint32_t ph = 0u;
@@ -241,6 +253,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         bool is_v;
         const int b = item(i, is_v);
         const int slot = b & 1;
+        if (is_v != pv_role) {  // the other issuer's item
+          if (++s == stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+          continue;
+        }
         if (!is_v) {
           // the score slot must have been read by the softmax of block b - 2
           if (b >= 2 && !wait_parity(smem_u32(&s_free[slot]), ((b - 2) >> 1) & 1, abort_flag)) {
@@ -292,9 +311,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           ph ^= 1u;
         }
       }
-      // every MMA issued by this thread is complete once final_bar flips
-      umma_commit(smem_u32(final_bar));
-      drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
+      // every MMA issued by this thread is complete once its final barrier flips
+      umma_commit(smem_u32(&final_bar[pv_role ? 1 : 0]));
+      drain_wait(smem_u32(&final_bar[pv_role ? 1 : 0]), 0, 50ull * 1000ull * 1000ull);
     }
     __syncwarp();
   } else {

@@ -603,9 +603,11 @@ tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& g
   chunks = chunks < 1 ? 1 : (chunks > p.nblk ? p.nblk : chunks);
   p.nb = (p.nblk + chunks - 1) / chunks;
   p.chunks = (p.nblk + p.nb - 1) / p.nb;
-  // a 3-deep ring of 32 KB stages at 16 query rows, 2-deep at 32, so two CTAs
-  // fit on an SM; TMEM: two score slots and two accumulators
-  p.stages = p.n_pad <= 16 ? 3 : 2;
+  // a 2-deep ring of 32 KB stages: in the load order K_0, K_1, V_0, K_2,
+  // V_1, ... the two MMA issuers (scores, P V) then each take their stage's
+  // fills in order (see attn_decode_kernel); TMEM: two score slots and two
+  // accumulators
+  p.stages = 2;
   p.tmem_cols = next_pow2(4 * p.n_pad < 32 ? 32 : 4 * p.n_pad);  // 2 score slots, 2 O's
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(tpb::kAttnHeadDim));
   const size_t rows = static_cast<size_t>(groups) * nkv * p.chunks * p.n_pad;
