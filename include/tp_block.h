@@ -392,7 +392,7 @@ tp_status tp_diag_bounded_wait(unsigned int limit_us, int* result, tp_stream_t s
  * Token count at or below which a call takes the weight-streaming (decode)
  * kernels instead of the tiled (prefill) kernels.  `max_tokens` in [0, 128];
  * 0 sends every call to the tiled kernels.  Process-wide; returns
- * TP_ERR_UNSUPPORTED for values outside the range.  The default is 64.
+ * TP_ERR_UNSUPPORTED for values outside the range.  The default is 128.
  */
 tp_status tp_set_decode_max_tokens(int max_tokens);
 int tp_get_decode_max_tokens(void);
