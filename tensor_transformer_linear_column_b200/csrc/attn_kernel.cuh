@@ -51,7 +51,7 @@ namespace tpb {
 
 constexpr int kAttnHeadDim = 128;
 constexpr int kAttnBlockKeys = 128;
-constexpr int kAttnMaxStages = 6;  // an even ring depth (the two MMA issuers rely on it)
+constexpr int kAttnMaxStages = 2;  // the two MMA issuers rely on exactly two (see below)
 // warp 0 TMA; warp 1 issues the score MMAs, warp 6 the P V MMAs; warps 2-5
 // softmax / epilogue
 constexpr int kAttnThreads = 224;
@@ -235,15 +235,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (lane == 0) {
       // ---------------- MMA issuers: warp 1 takes the K items (scores), warp 6
       // the V items (P V); both walk the load order to track ring stages.
-      // Item i is a K block for odd i and a V block for even i, except K_0
-      // (item 0) and the last item V_{nbc-1} (odd).  With an even ring depth a
-      // stage keeps the parity of its items, so an odd stage holds K blocks
-      // (and at most the last V) and an even stage V blocks (after K_0).
-      // Where a stage changes hands (K_0 -> a V, a K -> V_{nbc-1}), the P V
-      // issuer first waits for that V block's P, which needs every score up to
-      // that block, so the stage's previous fill has landed: a parity wait
-      // never matches an older phase.  The score MMAs so never queue behind a
-      // P V product that waits for its softmax.
+      // With two stages, stage 0 holds K_0 and then only V blocks, and stage 1
+      // only K blocks except the last item, V_{nbc-1}.  Where a stage changes
+      // hands (K_0 -> V_0, K_{nbc-1} -> V_{nbc-1}), the P V issuer waits for
+      // that block's P first, which needs the block's scores, so the previous
+      // fill has landed: a parity wait never matches an older phase.  The
+      // score MMAs so never queue behind a P V product that waits for its
+      // softmax.
       const bool pv_role = warp == 6;
       const uint32_t idesc_s = idesc_bf16_f32(128, kRows);               // K, Q both K-major
       const uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, false);  // V^T MN-major, P K-major

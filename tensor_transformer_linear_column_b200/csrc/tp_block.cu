@@ -571,7 +571,7 @@ tp_status run_linear_w8(const tp_bf16* x, const uint8_t* w8, const float* w_scal
 // only (not of the device), so the chunking and therefore the order of the
 // sums are the same on every GPU.  TP_ERR_UNSUPPORTED if G is not 1, 2, 4, 8
 // or 16.
-constexpr int kAttnTargetCtas = 148;  // one CTA per SM, one wave
+constexpr int kAttnTargetCtas = 296;  // two waves' worth of CTAs on 148 SMs
 
 tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& groups,
                     size_t& part_o_bytes, size_t& part_ml_bytes) {
@@ -599,18 +599,18 @@ tp_status plan_attn(int T, int past, int nq, int nkv, tpb::AttnParams& p, int& g
   }
   p.n_pad = p.Tq * G;
   p.nblk = (p.L + tpb::kAttnBlockKeys - 1) / tpb::kAttnBlockKeys;
-  // chunks per key-value head so the grid is about kAttnTargetCtas CTAs (one
+  // chunks per key-value head so the grid is about kAttnTargetCtas CTAs (two
   // per SM, one wave); every chunk streams nb blocks with a running softmax
   const int per_chunk = nkv * groups;  // CTAs per chunk index
   int chunks = (kAttnTargetCtas + per_chunk - 1) / per_chunk;
   chunks = chunks < 1 ? 1 : (chunks > p.nblk ? p.nblk : chunks);
   p.nb = (p.nblk + chunks - 1) / chunks;
   p.chunks = (p.nblk + p.nb - 1) / p.nb;
-  // one CTA per SM with a deep ring of 32 KB stages (6 at 16 query rows, 4 at
-  // 32), so up to three K and three V blocks are in flight; the depth is even
-  // so the two MMA issuers (scores, P V) each take their stages' fills in
-  // order (see attn_decode_kernel); TMEM: two score slots and two accumulators
-  p.stages = p.n_pad <= 16 ? 6 : 4;
+  // a 2-deep ring of 32 KB stages: in the load order K_0, K_1, V_0, K_2,
+  // V_1, ... the two MMA issuers (scores, P V) then each take their stage's
+  // fills in order (see attn_decode_kernel); TMEM: two score slots and two
+  // accumulators
+  p.stages = 2;
   p.tmem_cols = next_pow2(4 * p.n_pad < 32 ? 32 : 4 * p.n_pad);  // 2 score slots, 2 O's
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(tpb::kAttnHeadDim));
   const size_t rows = static_cast<size_t>(groups) * nkv * p.chunks * p.n_pad;
