@@ -112,6 +112,37 @@ __global__ void kv_append_kernel(const uint16_t* __restrict__ qkv, uint16_t* __r
   grid_launch_dependents();
 }
 
+// Reduce kRows per-lane values (one per query row) over the 32 lanes of a warp
+// with a transposing butterfly: at offset o a lane keeps the half of its rows
+// selected by bit o of its lane index and trades the other half with lane
+// ^ o, so kRows - 1 shuffles in total instead of 5 kRows.  On return v[0] holds
+// the warp's reduction of row ((lane >> 1) & 15) for kRows = 16 (lanes 2c and
+// 2c + 1 both hold row c), or of row `lane` for kRows = 32.
+template <int kRows, bool kMax>
+__device__ __forceinline__ float warp_rows_reduce(float (&v)[kRows], int lane) {
+  int n = kRows;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < kRows / 2; ++i) {
+        if (i < n / 2) {
+          const float send = upper ? v[i] : v[i + n / 2];
+          const float keep = upper ? v[i + n / 2] : v[i];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+          v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+      }
+      n >>= 1;
+    } else {
+      const float recv = __shfl_xor_sync(0xffffffffu, v[0], o);
+      v[0] = kMax ? fmaxf(v[0], recv) : v[0] + recv;
+    }
+  }
+  return v[0];
+}
+
 // Two CTAs per SM (the ring of one overlaps the softmax of the other): at most
 // 170 registers per thread.  kRows = n_pad (16 or 32).
 template <int kRows>
@@ -364,13 +395,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
       for (int j = 0; j < kRows; ++j)
         sc[j] = key <= lim[j] ? __uint_as_float(v[j]) * p.scale_log2 : neg_inf();
-      // the block maximum per row: warp butterfly, then the four warps
+      // the block maximum per row: a transposing warp butterfly, then the four
+      // warps in order
+      const int my_row = kRows == 32 ? lane : (lane >> 1) & 15;
+      {
+        float mx[kRows];
 #pragma unroll
-      for (int j = 0; j < kRows; ++j) {
-        float mx = sc[j];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) red_m[q4 * 32 + j] = mx;
+        for (int j = 0; j < kRows; ++j) mx[j] = sc[j];
+        const float m = warp_rows_reduce<kRows, true>(mx, lane);
+        if (kRows == 32 || (lane & 1) == 0) red_m[q4 * 32 + my_row] = m;
       }
       named_barrier_sync(1, 128);
       float* ms = m_s + slot * 32;  // accumulator b % 2's running state
@@ -389,16 +422,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[slot]),
                                                        ((b - 2) >> 1) & 1, abort_flag));
       uint8_t* pslot = ps + static_cast<size_t>(slot) * 2u * kQHalf + static_cast<size_t>(r >> 6) * kQHalf;
+      {
+        float pr[kRows];
 #pragma unroll
-      for (int j = 0; j < kRows; ++j) {
-        const float m = ms[j];
-        const float e = sc[j] == neg_inf() ? 0.0f : exp2f(sc[j] - m);
-        const __nv_bfloat16 hb = __float2bfloat16_rn(e);
-        *reinterpret_cast<__nv_bfloat16*>(pslot + j * 128 + ((kc ^ (j & 7)) << 4) + kw) = hb;
-        float sm = __bfloat162float(hb);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-        if (lane == 0) red_s[q4 * 32 + j] = sm;
+        for (int j = 0; j < kRows; ++j) {
+          const float m = ms[j];
+          const float e = sc[j] == neg_inf() ? 0.0f : exp2f(sc[j] - m);
+          const __nv_bfloat16 hb = __float2bfloat16_rn(e);
+          *reinterpret_cast<__nv_bfloat16*>(pslot + j * 128 + ((kc ^ (j & 7)) << 4) + kw) = hb;
+          pr[j] = __bfloat162float(hb);
+        }
+        const float sm = warp_rows_reduce<kRows, false>(pr, lane);
+        if (kRows == 32 || (lane & 1) == 0) red_s[q4 * 32 + my_row] = sm;
       }
       named_barrier_sync(1, 128);
       if (et < kRows)
