@@ -423,14 +423,30 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                                                        ((b - 2) >> 1) & 1, abort_flag));
       uint8_t* pslot = ps + static_cast<size_t>(slot) * 2u * kQHalf + static_cast<size_t>(r >> 6) * kQHalf;
       {
+        // p of rows j (this lane's key) as bf16; lanes 2m and 2m + 1 (keys
+        // 2m, 2m + 1) then trade one value per row pair so that each writes one
+        // 4-byte word: the even lane row j, the odd lane row j + 1
         float pr[kRows];
+        uint16_t pb16[kRows];
 #pragma unroll
         for (int j = 0; j < kRows; ++j) {
           const float m = ms[j];
           const float e = sc[j] == neg_inf() ? 0.0f : exp2f(sc[j] - m);
           const __nv_bfloat16 hb = __float2bfloat16_rn(e);
-          *reinterpret_cast<__nv_bfloat16*>(pslot + j * 128 + ((kc ^ (j & 7)) << 4) + kw) = hb;
+          pb16[j] = *reinterpret_cast<const uint16_t*>(&hb);
           pr[j] = __bfloat162float(hb);
+        }
+        const bool odd = (lane & 1) != 0;
+        const int kw4 = kw & ~3;  // the word of keys 2m, 2m + 1
+#pragma unroll
+        for (int j = 0; j < kRows; j += 2) {
+          // even lane sends its row j + 1 value, odd lane its row j value
+          const uint32_t give = odd ? pb16[j] : pb16[j + 1];
+          const uint32_t got = __shfl_xor_sync(0xffffffffu, give, 1);
+          const int row = odd ? j + 1 : j;
+          const uint32_t word = odd ? (got | (static_cast<uint32_t>(pb16[j + 1]) << 16))
+                                    : (static_cast<uint32_t>(pb16[j]) | (got << 16));
+          *reinterpret_cast<uint32_t*>(pslot + row * 128 + ((kc ^ (row & 7)) << 4) + kw4) = word;
         }
         const float sm = warp_rows_reduce<kRows, false>(pr, lane);
         if (kRows == 32 || (lane & 1) == 0) red_s[q4 * 32 + my_row] = sm;
@@ -517,9 +533,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
-// One warp per (token i, query head h): merge the chunk partials of head h in
-// chunk order.  M = max_c m_c; ctx = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c,
-// one bf16 rounding.  Lane l owns d = 4 l .. 4 l + 3.
+// One warp per (token i, query head h): merge the chunk partials of head h.
+// M = max_c m_c; ctx = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c, one bf16
+// rounding.  The maximum and the sum of the l_c are taken across the lanes
+// (chunk c on lane c % 32, then a fixed butterfly); the weighted sum of the
+// o_c runs over the chunks in order, four loads in flight.  Lane l owns
+// d = 4 l .. 4 l + 3.  Every order is fixed, so the result is bit-identical
+// from run to run.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o,
                                     const float* __restrict__ part_ml, int T, int nq, int nkv,
                                     int G, int Tq, int n_pad, int chunks,
@@ -534,21 +554,31 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   const int grp = i / Tq;
   const int n = (i - grp * Tq) * G + (h - g * G);
   const size_t base = (static_cast<size_t>(grp) * nkv + g) * chunks;
+  const float* ml = part_ml + (base * n_pad + n) * 2;  // chunk c at ml[c * n_pad * 2]
+  const size_t ml_stride = static_cast<size_t>(n_pad) * 2;
   float M = neg_inf();
-  for (int c = 0; c < chunks; ++c)
-    M = fmaxf(M, part_ml[((base + c) * n_pad + n) * 2]);
+  for (int c = lane; c < chunks; c += 32) M = fmaxf(M, __ldg(ml + c * ml_stride));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.0f;
+  for (int c = lane; c < chunks; c += 32) {
+    const float m = __ldg(ml + c * ml_stride);
+    if (m != neg_inf()) L = fmaf(exp2f(m - M), __ldg(ml + c * ml_stride + 1), L);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float* po = part_o + (base * n_pad + n) * kAttnHeadDim + 4 * lane;
+  const size_t o_stride = static_cast<size_t>(n_pad) * kAttnHeadDim;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int c = 0; c < chunks; ++c) {
-    const float m = part_ml[((base + c) * n_pad + n) * 2];
+    const float m = __ldg(ml + c * ml_stride);
     const float w = m == neg_inf() ? 0.0f : exp2f(m - M);
-    L += w * part_ml[((base + c) * n_pad + n) * 2 + 1];
-    const float4 o = *reinterpret_cast<const float4*>(
-        part_o + ((base + c) * n_pad + n) * kAttnHeadDim + 4 * lane);
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
+    const float4 o = __ldg(reinterpret_cast<const float4*>(po + c * o_stride));
+    acc.x = fmaf(w, o.x, acc.x);
+    acc.y = fmaf(w, o.y, acc.y);
+    acc.z = fmaf(w, o.z, acc.z);
+    acc.w = fmaf(w, o.w, acc.w);
   }
   const float inv = 1.0f / L;
   uint2 packed;
