@@ -12,12 +12,12 @@
 // What is computed (grouped-query causal attention, scores q.k / sqrt(d)):
 // query head h reads key-value head g = h / G (G = nq / nkv); new token i sits
 // at position past + i and sees cached keys 0 .. past + i.  The kernels:
-//   kv_append_kernel      copies the new tokens' K and V from qkv into the
-//                         cache rows [past, past + T);
 //   attn_decode_kernel    CTA (chunk c, key-value head g, token group z):
 //                         keys [c C, (c + 1) C) of head g against the queries
 //                         of its G heads x Tq tokens; writes an unnormalised
-//                         partial (running max m, sum l, sum of p v);
+//                         partial (running max m, sum l, sum of p v).  The
+//                         CTAs whose chunk holds rows [past, past + T) first
+//                         copy the new tokens' K and V from qkv into them;
 //   attn_combine_kernel   per (token, query head): the partials of all chunks
 //                         merged in chunk order, divided by the total sum.
 //
@@ -74,7 +74,19 @@ struct AttnParams {
   float scale_log2;  // log2(e) / sqrt(d)
   float* part_o;  // [groups][nkv][chunks][n_pad][d] unnormalised sums of p v
   float* part_ml; // [groups][nkv][chunks][n_pad][2]  (max m, sum l) in base-2 units
+  // the new tokens' keys and values, copied into the caches by the CTAs whose
+  // chunk holds rows [past, past + T)
+  const uint16_t* qkv;  // [T, (nq + 2 nkv) d]
+  uint16_t* k_cache;    // [nkv, max_len, d]
+  uint16_t* v_cache;
+  int max_len;
 };
+
+// Order this thread's generic-proxy global writes before later async-proxy
+// (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // Shared memory (dynamic, base rounded up to 1024 B): ring [stages][32 KB],
 // Q [2 d halves][n_pad][64] bf16, P [2 slots][2 key halves][n_pad][64] bf16,
@@ -84,32 +96,6 @@ __host__ __device__ inline int attn_q_bytes(int n_pad) { return n_pad * kAttnHea
 __host__ __device__ inline int attn_smem_bytes(int stages, int n_pad) {
   return 1024 + stages * kAttnBlockBytes + 3 * attn_q_bytes(n_pad) + 2 * 4 * 32 * 4 + 5 * 32 * 4 +
          (2 * kAttnMaxStages + 11) * 8 + 16;
-}
-
-// Copy the new tokens' keys and values into the cache: for token i and
-// key-value head g, qkv[i, (nq + g) d ..] -> k_cache[g, past + i, :] and
-// qkv[i, (nq + nkv + g) d ..] -> v_cache[g, past + i, :], 16 bytes per thread.
-__global__ void kv_append_kernel(const uint16_t* __restrict__ qkv, uint16_t* __restrict__ kc,
-                                 uint16_t* __restrict__ vc, int T, int past, int max_len, int nq,
-                                 int nkv) {
-  grid_dependency_wait();  // qkv comes from the preceding kernel
-  constexpr int kVec = kAttnHeadDim / 8;  // 16-byte pieces per head row
-  const int total = T * nkv * kVec * 2;
-  const size_t ld = static_cast<size_t>(nq + 2 * nkv) * kAttnHeadDim;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int piece = e % kVec;
-    const int rest = e / kVec;
-    const int g = rest % nkv;
-    const int which = (rest / nkv) & 1;  // 0 = K, 1 = V
-    const int i = rest / (2 * nkv);
-    const uint4* src = reinterpret_cast<const uint4*>(
-        qkv + static_cast<size_t>(i) * ld + static_cast<size_t>(nq + which * nkv + g) * kAttnHeadDim) + piece;
-    uint16_t* cache = which ? vc : kc;
-    uint4* dst = reinterpret_cast<uint4*>(
-        cache + (static_cast<size_t>(g) * max_len + past + i) * kAttnHeadDim) + piece;
-    *dst = *src;
-  }
-  grid_launch_dependents();
 }
 
 // Reduce kRows per-lane values (one per query row) over the 32 lanes of a warp
@@ -223,12 +209,37 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   };
 
   if (warp == 0) {
+    // ---------------- the new tokens' K and V rows of head g that fall in this
+    // chunk go into the caches first (the whole warp, 16 bytes per lane per
+    // step), then the warp's writes are ordered before the TMA loads of them
+    grid_dependency_wait();  // qkv comes from the preceding kernel
+    {
+      const int r0 = key0 > p.past ? key0 : p.past;
+      const int kend = key0 + nbc * kAttnBlockKeys;
+      const int r1 = kend < p.L ? kend : p.L;
+      constexpr int kVec = kAttnHeadDim / 8;  // 16-byte pieces of a head row
+      const size_t ld = static_cast<size_t>(p.nq + 2 * p.nkv) * kAttnHeadDim;
+      for (int e = lane; e < (r1 - r0) * kVec * 2; e += 32) {
+        const int piece = e % kVec;
+        const int which = (e / kVec) & 1;  // 0 = K, 1 = V
+        const int row = r0 + e / (2 * kVec);
+        const int tok = row - p.past;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.qkv + static_cast<size_t>(tok) * ld +
+            static_cast<size_t>(p.nq + which * p.nkv + g) * kAttnHeadDim) + piece;
+        uint16_t* cache = which ? p.v_cache : p.k_cache;
+        uint4* dst = reinterpret_cast<uint4*>(
+            cache + (static_cast<size_t>(g) * p.max_len + row) * kAttnHeadDim) + piece;
+        *dst = __ldg(src);
+      }
+      fence_proxy_async_global();
+      __syncwarp();
+    }
     if (lane == 0) {
       // ---------------- TMA producer
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
-      grid_dependency_wait();  // qkv and the appended cache rows come from preceding kernels
       const uint32_t qb = smem_u32(q_bar);
       mbar_arrive_expect_tx(qb, 2u * kQHalf);
       tma_load_3d(smem_u32(qs), &tmap_q, qb, 0, g * p.G, tok0);

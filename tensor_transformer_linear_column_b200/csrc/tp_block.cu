@@ -842,23 +842,14 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                        static_cast<uint64_t>(max_len) * head_dim, tpb::kAttnBlockKeys, 1))
     return TP_ERR_CUDA;
 
+  p.qkv = qkv;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.max_len = max_len;
   cudaLaunchAttribute attr[1];
   const int nattr = launch_attrs(attr, 0);
-  // 1. the new tokens' keys and values into the cache
-  {
-    const int total = T * n_kv_heads * (tpb::kAttnHeadDim / 8) * 2;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>((total + 255) / 256), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = static_cast<unsigned>(nattr);
-    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::kv_append_kernel, qkv, k_cache, v_cache, T, past,
-                                    max_len, n_q_heads, n_kv_heads),
-                 "launch kv_append_kernel"))
-      return TP_ERR_CUDA;
-  }
-  // 2. chunk partials: grid (chunks, key-value heads, token groups)
+  // 1. chunk partials: grid (chunks, key-value heads, token groups); the CTAs
+  //    holding rows [past, past + T) write the new keys and values first
   {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(p.chunks), static_cast<unsigned>(n_kv_heads),
@@ -873,7 +864,7 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                               : cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel<32>, tq, tk, tv, p);
     if (!cuda_ok(e, "launch attn_decode_kernel")) return TP_ERR_CUDA;
   }
-  // 3. merge the chunks of every (token, query head) in chunk order
+  // 2. merge the chunks of every (token, query head)
   {
     const int warps = T * n_q_heads;
     cudaLaunchConfig_t cfg{};
