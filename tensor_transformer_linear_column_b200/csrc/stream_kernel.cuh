@@ -58,8 +58,7 @@
 // and store the bf16 tile straight into tensor memory, one row per thread, as
 // the MMA's A operand.  So per k-block shared memory carries only the codes
 // (written by TMA, read once) and x, not a bf16 tile written and read again.
-// Four to eight TMEM A slots (the columns the accumulators leave) decouple
-// conversion from the MMAs: a slot is refilled only once its MMAs complete.  The row scale
+// Four TMEM A slots decouple conversion from the MMAs.  The row scale
 // multiplies the fp32 sum before bias and activation; HBM traffic is halved.
 //
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
@@ -84,8 +83,7 @@ struct StreamParams {
   int tmem_cols;  // columns of one TMEM region (power of two >= max(32, t_pad))
   int kpb;        // k-blocks per TMA box and pipeline stage (1 or 2)
   int l2_ahead;   // boxes after the ring's first fill prefetched into L2 before the grid wait
-  int stages;     // smem pipeline depth (<= 8; 8-bit weights: even, <= 12)
-  int w8_slots;   // 8-bit weights: TMEM A slots (even, 4..8): the TMEM the accumulators leave
+  int stages;     // smem pipeline depth (<= 8)
   int stage_bytes;
   int act;        // tp_act
   int prefetch_w; // weights may be read before the preceding grid completes
@@ -108,14 +106,12 @@ constexpr int kStreamMaxStages = 8;
 constexpr int kStreamMaxStagesW8 = 12;  // 8 KB code stages: a deeper ring in the same memory
 constexpr int kStreamReleaseBack = 2;  // boxes still to issue when the next grid is released
 constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when spc > 1
-constexpr int kStreamW8MinSlots = 4;  // 8-bit weights: bf16 k-blocks in TMEM (A operand slots)
-constexpr int kStreamW8MaxSlots = 8;
+constexpr int kStreamW8Slots = 4;   // 8-bit weights: bf16 k-blocks in TMEM (A operand slots)
 
 // TMEM columns a CTA allocates: two accumulator regions of tmem_cols each,
-// and with 8-bit weights at least four 32-column A slots (the power-of-two
-// allocation's remaining columns become more slots, up to eight).
+// and with 8-bit weights four 32-column A slots.
 __host__ __device__ inline int stream_tmem_alloc_cols(int tmem_cols, bool w8) {
-  const int need = 2 * tmem_cols + (w8 ? kStreamW8MinSlots * 32 : 0);
+  const int need = 2 * tmem_cols + (w8 ? kStreamW8Slots * 32 : 0);
   int c = 32;
   while (c < need) c <<= 1;
   return c;
@@ -128,7 +124,7 @@ __host__ __device__ inline int stream_tmem_alloc_cols(int tmem_cols, bool w8) {
 //                               (64-byte swizzle), converted into TMEM
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
-//   a_full[8], a_empty[8] (8-bit weights: TMEM A slots), tmem slot, abort flag
+//   a_full[4], a_empty[4] (8-bit weights: TMEM A slots), tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
 //
 // Row stride RS of the receive buffer: T rounded up to 4 floats (one 16-byte
@@ -151,7 +147,7 @@ __host__ __device__ inline int stream_data_bytes(int stages, int stage_bytes, in
 // seg_empty[2], final[2], recv, then `stream_extra_bars` more: a_full[4] and
 // a_empty[4] with 8-bit weights, an unused [stages] otherwise.
 __host__ __device__ inline int stream_extra_bars(int stages, bool w8) {
-  return w8 ? 2 * kStreamW8MaxSlots : stages;
+  return w8 ? 2 * kStreamW8Slots : stages;
 }
 
 __host__ inline int stream_smem_bytes(int stages, int stage_bytes, int T, int csize, bool w8) {
@@ -211,7 +207,7 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
 // t = 32 quarter + lane = weight row t of the tile: it reads its row's 64
 // codes (four 16-byte chunks; chunk c sits at chunk c ^ ((t / 2) % 4) of the
 // row under the 64-byte swizzle), converts them and stores the 64 bf16 values
-// as 32 columns of A slot i % w8_slots.  Every warp takes every box of its group in
+// as 32 columns of A slot i % 4.  Every warp takes every box of its group in
 // order and arrives for it whatever its waits returned, so the arrivals stay
 // matched.
 __device__ __forceinline__ void stream_convert_w8(const StreamParams& p, uint8_t* smem,
@@ -226,8 +222,8 @@ __device__ __forceinline__ void stream_convert_w8(const StreamParams& p, uint8_t
   for (int i = group; i < nbox; i += 2) {
     const int s = i % p.stages;
     const uint32_t ph = static_cast<uint32_t>(i / p.stages) & 1u;
-    const int a = i % p.w8_slots;
-    const uint32_t aph = static_cast<uint32_t>(i / p.w8_slots) & 1u;
+    const int a = i & (kStreamW8Slots - 1);
+    const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
     ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
     ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
     // the warp stores only when all its lanes' waits succeeded (the store is
@@ -279,8 +275,8 @@ __global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8
   uint64_t* seg_empty = bars + 2 * p.stages + 2;  // [2]
   uint64_t* final_bar = bars + 2 * p.stages + 4;  // [2], one per MMA issuer
   uint64_t* recv_bar = bars + 2 * p.stages + 6;   // bytes of the peers' partials for my rows
-  uint64_t* a_full = bars + 2 * p.stages + 7;     // [8]: 8-bit weights, A slot converted (4 warps)
-  uint64_t* a_empty = a_full + kStreamW8MaxSlots; // [8]: A slot read by the MMAs (commit)
+  uint64_t* a_full = bars + 2 * p.stages + 7;     // [4]: 8-bit weights, A slot converted (4 warps)
+  uint64_t* a_empty = a_full + kStreamW8Slots;    // [4]: A slot read by the MMAs (commit)
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(bars + 2 * p.stages + 7 + stream_extra_bars(p.stages, kW8));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -311,7 +307,7 @@ __global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     if constexpr (kW8) {
-      for (int a = 0; a < p.w8_slots; ++a) {
+      for (int a = 0; a < kStreamW8Slots; ++a) {
         mbar_init(smem_u32(&a_full[a]), 4);  // one arrive per converting warp
         mbar_init(smem_u32(&a_empty[a]), 1);
       }
@@ -455,8 +451,8 @@ __global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8
         bool first = true;
         for (; i < end; ++i) {
           if (kShards || (s & 1) == me) {
-            const int a = kW8 ? i % p.w8_slots : 0;
-            const uint32_t aph = kW8 ? static_cast<uint32_t>(i / p.w8_slots) & 1u : 0u;
+            const int a = i & (kStreamW8Slots - 1);
+            const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
             if (!wait_parity(smem_u32(kW8 ? &a_full[a] : &full_bar[s]), kW8 ? aph : ph,
                              abort_flag)) {
               ok = false;

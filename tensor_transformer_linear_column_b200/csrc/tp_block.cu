@@ -337,12 +337,6 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
          tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8) > max_smem)
     p.stages -= w8 ? 2 : 1;  // 8-bit weights keep an even depth
   smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8);
-  // 8-bit weights: every 32 columns the accumulators leave of the allocation
-  // hold one more A slot (an even count, so the converter groups never share)
-  if (w8) {
-    const int slots = (tpb::stream_tmem_alloc_cols(p.tmem_cols, true) - 2 * p.tmem_cols) / 32;
-    p.w8_slots = (slots > tpb::kStreamW8MaxSlots ? tpb::kStreamW8MaxSlots : slots) & ~1;
-  }
   // The CTAs that share an SM must fit their TMEM allocations together: a CTA
   // whose allocation waited for a cluster peer on the same SM to finish would
   // wait for ever (the peer waits for it at the cluster barrier).  Shared
