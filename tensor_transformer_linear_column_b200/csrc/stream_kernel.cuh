@@ -93,9 +93,6 @@ struct StreamParams {
 };
 
 constexpr int kStreamThreads = 224;
-// 8-bit weights: four more warps (7-10) convert the odd boxes while warps 0-3
-// convert the even ones
-constexpr int kStreamThreadsW8 = 352;
 constexpr int kStreamProducerWarp = 4;
 constexpr int kStreamMmaWarp = 5;   // MMA issuers: warps 5 and 6
 constexpr int kStreamMmaWarps = 2;
@@ -201,53 +198,6 @@ __host__ __device__ inline void stream_cta_range(const StreamParams& p, int cran
   }
 }
 
-// 8-bit weights: convert the boxes i with i % 2 == group (two converter groups
-// of four warps; the even ring depth makes every stage belong to one group).
-// The thread of lane quarter `quarter` and lane `lane` owns TMEM lane
-// t = 32 quarter + lane = weight row t of the tile: it reads its row's 64
-// codes (four 16-byte chunks; chunk c sits at chunk c ^ ((t / 2) % 4) of the
-// row under the 64-byte swizzle), converts them and stores the 64 bf16 values
-// as 32 columns of A slot i % 4.  Every warp takes every box of its group in
-// order and arrives for it whatever its waits returned, so the arrivals stay
-// matched.
-__device__ __forceinline__ void stream_convert_w8(const StreamParams& p, uint8_t* smem,
-                                                  uint64_t* full_bar, uint64_t* a_full,
-                                                  uint64_t* a_empty, uint32_t a_base, int nbox,
-                                                  int group, int quarter, int lane,
-                                                  volatile int* abort_flag) {
-  const int t = quarter * 32 + lane;
-  const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-  const int sw = (t >> 1) & 3;
-  bool ok = true;
-  for (int i = group; i < nbox; i += 2) {
-    const int s = i % p.stages;
-    const uint32_t ph = static_cast<uint32_t>(i / p.stages) & 1u;
-    const int a = i & (kStreamW8Slots - 1);
-    const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
-    ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
-    ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
-    // the warp stores only when all its lanes' waits succeeded (the store is
-    // warp-wide)
-    if (__all_sync(0xffffffffu, ok)) {
-      const uint8_t* row = smem + s * p.stage_bytes + t * kStreamTileK;
-      uint32_t w[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 q = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
-        const uint4 lo = e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
-        const uint4 hi = e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
-        w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
-        w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
-      }
-      tmem_st32(a_base + lane_addr + static_cast<uint32_t>(a * 32), w);
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&a_full[a]));
-  }
-}
-
 // Registers are granted to a CTA per group of four warps, so the seven-warp
 // CTA is charged as eight; the bounds below are stated for 256 threads to make
 // the compiler budget for that.  kShards = false: one accumulation segment per CTA
@@ -256,10 +206,8 @@ __device__ __forceinline__ void stream_convert_w8(const StreamParams& p, uint8_t
 // kShards = true: several shards per CTA (spc > 1) folded in a register
 // running sum, at most 128 registers (two CTAs per SM).
 constexpr int kStreamRegThreads = 256;
-// With 8-bit weights (eleven warps, counted as twelve) two CTAs per SM: at most
-// 85 registers per thread.
 template <bool kShards, bool kW8>
-__global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8) ? 2 : 3)
+__global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
     stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_x, const StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -411,13 +359,6 @@ __global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8
       }
     }
     __syncwarp();
-  } else if (warp >= kStreamMmaWarp + kStreamMmaWarps) {
-    // ---------------- warps 7-10 (8-bit weights only): the odd boxes
-    if constexpr (kW8)
-      stream_convert_w8(p, smem, full_bar, a_full, a_empty, tmem_d + a_col0, nbox, 1, warp & 3,
-                        lane, abort_flag);
-    __syncwarp();
-    if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else if (warp >= kStreamMmaWarp) {
     const int me = warp - kStreamMmaWarp;  // issuer 0 or 1
     if (lane == 0 && (!kShards || me == 0)) {
@@ -502,9 +443,48 @@ __global__ void __launch_bounds__(kW8 ? 384 : kStreamRegThreads, (kShards || kW8
     if (multi) cluster_wait_acquire();  // phase 1 (these warps send nothing)
   } else {
     if constexpr (kW8) {
-      // ---------------- warps 0-3, first: the even boxes' E4M3 -> bf16 into TMEM
-      stream_convert_w8(p, smem, full_bar, a_full, a_empty, tmem_d + a_col0, nbox, 0, warp, lane,
-                        abort_flag);
+      // ---------------- warps 0-3, first: E4M3 -> bf16 into TMEM.  Thread t
+      // owns TMEM lane t = weight row t of the tile: it reads its row's 64
+      // codes (four 16-byte chunks; chunk c sits at chunk c ^ ((t / 2) % 4) of
+      // the row under the 64-byte swizzle), converts them and stores the 64
+      // bf16 values as 32 columns of A slot i % 4.  Every converter thread
+      // takes every box in order, whatever its waits returned, so the warps'
+      // arrivals stay matched.
+      const int t = static_cast<int>(threadIdx.x);
+      const uint32_t lane_addr_c = static_cast<uint32_t>(warp * 32) << 16;
+      const int sw = (t >> 1) & 3;
+      int s = 0;
+      uint32_t ph = 0u;
+      bool ok = true;
+      for (int i = 0; i < nbox; ++i) {
+        const int a = i & (kStreamW8Slots - 1);
+        const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
+        ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
+        ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
+        // the warp stores only when all its lanes' waits succeeded (the store
+        // is warp-wide); every warp arrives for every box whatever happened
+        if (__all_sync(0xffffffffu, ok)) {
+          const uint8_t* row = smem + s * p.stage_bytes + t * kStreamTileK;
+          uint32_t w[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+            const uint4 lo = e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
+            const uint4 hi = e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
+            w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+            w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+          }
+          tmem_st32(tmem_d + lane_addr_c + a_col0 + static_cast<uint32_t>(a * 32), w);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&a_full[a]));
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
     }
     // ---------------- warps 0-3: drain TMEM, fold shards in order, send rows to their owners
     grid_dependency_wait();

@@ -322,9 +322,6 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
     int stages = kbs / p.kpb;
     const int max_stages = w8 ? tpb::kStreamMaxStagesW8 : tpb::kStreamMaxStages;
     stages = stages < 2 ? 2 : (stages > max_stages ? max_stages : stages);
-    // 8-bit weights: an even depth, so each stage's boxes all belong to one
-    // converter group (boxes alternate between the two groups)
-    if (w8) stages &= ~1;
     p.stages = stages;
     p.stage_bytes = p.kpb * kb_bytes;
     // short streams: two more boxes into L2 before the grid wait (measured
@@ -335,7 +332,7 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
   // large T: the receive buffer leaves room for two stages only
   while (p.stages > 2 &&
          tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8) > max_smem)
-    p.stages -= w8 ? 2 : 1;  // 8-bit weights keep an even depth
+    --p.stages;
   smem = tpb::stream_smem_bytes(p.stages, p.stage_bytes, p.T, p.csize, w8);
   // The CTAs that share an SM must fit their TMEM allocations together: a CTA
   // whose allocation waited for a cluster peer on the same SM to finish would
@@ -383,7 +380,7 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(n_tiles), static_cast<unsigned>(p.csize), 1);
-  cfg.blockDim = dim3(w8 ? tpb::kStreamThreadsW8 : tpb::kStreamThreads, 1, 1);
+  cfg.blockDim = dim3(tpb::kStreamThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
