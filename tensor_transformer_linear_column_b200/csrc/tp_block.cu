@@ -901,8 +901,12 @@ tp_status tp_sp_add_rmsnorm(const tp_bf16* y, const tp_bf16* residual, const tp_
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cfg.attrs = attr;
   cfg.numAttrs = static_cast<unsigned>(launch_attrs(attr, 0));
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, tpb::add_rmsnorm_kernel, y, residual, gamma, H,
-                                           eps, r_out, n_out);
+  const bool in_regs = H <= tpb::kNormThreads * tpb::kNormVecPerThread * 8;
+  const cudaError_t e =
+      in_regs ? cudaLaunchKernelEx(&cfg, tpb::add_rmsnorm_kernel<true>, y, residual, gamma, H, eps,
+                                   r_out, n_out)
+              : cudaLaunchKernelEx(&cfg, tpb::add_rmsnorm_kernel<false>, y, residual, gamma, H, eps,
+                                   r_out, n_out);
   return cuda_ok(e, "launch add_rmsnorm_kernel") ? TP_OK : TP_ERR_CUDA;
 }
 
