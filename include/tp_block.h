@@ -252,6 +252,37 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                          tp_stream_t stream);
 
 /*
+ * The same attention core as tp_attn_decode (same sharding, same causal
+ * grouped-query operation, same cache update), for many new tokens at once: a
+ * prompt (past = 0) or a chunk of one appended after `past` cached tokens.
+ * The queries of one head fill 128-row tiles; each tile streams the keys and
+ * values it may see once, with a running softmax, and needs no workspace.
+ *   1. the new tokens' keys and values (columns K and V of qkv) are written
+ *      into the cache at positions [past, past + T);
+ *   2. ctx[i, h d .. h d + d) = sum_j p_j v_j over keys j <= past + i of
+ *      key-value head h / (nq / nkv), p = softmax_j(q_i,h . k_j / sqrt(d)).
+ * Arithmetic: bf16 q, k, v; scores, maxima and sums in fp32; the softmax
+ * weights are rounded to bf16 for the weighted sum of v (fp32 accumulate) and
+ * their row sum is taken from the fp32 weights before that rounding.  The
+ * running maximum is raised only when a block of 128 keys exceeds it by more
+ * than a factor 2^8, so the weights lie in [0, 2^8] before normalisation.
+ * The key blocks of a row are visited in ascending order by one CTA, so the
+ * result is bit-identical from run to run.
+ *   qkv      [T, (nq + 2 nkv) d]  tp_attn_proj_forward's qkv_out   (read)
+ *   k_cache  [nkv, max_len, d]    rows [0, past) hold the cached keys;
+ *                                 rows [past, past + T) are written
+ *   v_cache  [nkv, max_len, d]    likewise for values
+ *   ctx      [T, nq d]            the input of the output projection (written)
+ * Requires head_dim == 128 (else TP_ERR_UNSUPPORTED), nq a multiple of nkv and
+ * past + T <= max_len (else TP_ERR_SHAPE), and t dividing both head counts
+ * (else TP_ERR_TP_DEGREE).  Calls that overlap on the GPU must not share a
+ * cache.
+ */
+tp_status tp_attn_prefill(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache, int T,
+                          int past, int max_len, int n_q_heads, int n_kv_heads, int head_dim,
+                          int tp_degree, tp_bf16* ctx, tp_stream_t stream);
+
+/*
  * The sequence-parallel region after a row-parallel linear: residual add and
  * RMSNorm, token shard by token shard.  Sequence parallelism splits the parts
  * of a layer that tensor parallelism leaves whole (normalisation, dropout)

@@ -49,6 +49,7 @@ SIGNATURES = {
     "tp_attn_decode_workspace_bytes": (_Z, [_I, _I, _I, _I, _I]),
     "tp_sp_add_rmsnorm": (_I, [_P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
     "tp_attn_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "tp_attn_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "tp_mlp_backward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
                              _P]),
     "tp_colpar_gemm_gelu_w8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
@@ -433,6 +434,31 @@ def tp_attn_decode(qkv: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
                                _ptr(ctx, "ctx", dev), workspace.data_ptr(),
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "tp_attn_decode")
+    return ctx
+
+
+def tp_attn_prefill(qkv: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, past: int,
+                    n_q_heads: int, n_kv_heads: int, head_dim: int, tp_degree: int,
+                    ctx: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The attention core for many new tokens at once (a prompt or a chunk of
+    one): ctx [T, nq d] of qkv [T, (nq + 2 nkv) d] over the caches k_cache,
+    v_cache [nkv, max_len, d] holding `past` tokens; appends the new tokens'
+    keys and values to the caches in place.  Needs no workspace."""
+    T = qkv.shape[0]
+    if qkv.shape[1] != (n_q_heads + 2 * n_kv_heads) * head_dim:
+        raise ValueError("qkv must be [T, (nq + 2 nkv) d]")
+    if k_cache.dim() != 3 or tuple(k_cache.shape) != tuple(v_cache.shape) or \
+            k_cache.shape[0] != n_kv_heads or k_cache.shape[2] != head_dim:
+        raise ValueError("caches must be [nkv, max_len, d]")
+    dev = _device(qkv)
+    if ctx is None:
+        ctx = torch.empty((T, n_q_heads * head_dim), dtype=torch.bfloat16, device=dev)
+    st = load().tp_attn_prefill(_ptr(qkv, "qkv", dev), _ptr(k_cache, "k_cache", dev),
+                                _ptr(v_cache, "v_cache", dev), T, int(past), k_cache.shape[1],
+                                int(n_q_heads), int(n_kv_heads), int(head_dim), int(tp_degree),
+                                _ptr(ctx, "ctx", dev), _stream(stream))
+    _check(st, "tp_attn_prefill")
     return ctx
 
 

@@ -1,0 +1,333 @@
+// attn_prefill_kernel.cuh -- the attention core when many tokens arrive at
+// once (a prompt, or a long chunk of one appended to a cache): every query row
+// of a head attends over the keys it may see, 128 query rows per CTA.
+//
+// Same operation as attn_decode_kernel (grouped-query causal attention, scores
+// q.k / sqrt(d), query head h reads key-value head h / G, new token i at
+// position past + i sees keys 0 .. past + i), with the heads split across the
+// tensor-parallel shards and no exchange (xingyuzhitong.com "Tensor vs
+// Pipeline Parallelism", section "Tensor parallelism: split inside each
+// layer").  The decode kernel puts keys on the MMA's M side because a decode
+// step has few query rows; here the queries fill M = 128 and each softmax
+// thread owns one query row, so the row maximum and sum need no shuffles.
+//
+// Kernels:
+//   kv_append_kernel      copies the new tokens' K and V (columns of qkv) into
+//                         rows [past, past + T) of the caches;
+//   attn_prefill_kernel   CTA (query head h, tile of 128 new tokens); key
+//                         blocks of 128 from 0 up to the tile's last visible
+//                         key, each block:
+//     S = Q K_b^T            tcgen05.mma into TMEM columns [0, 128), fp32
+//     softmax (warps 0-3)    thread r = query row r: masks keys past its
+//                            position (the diagonal blocks only), takes the
+//                            block maximum, p = 2^(s log2(e)/sqrt(d) - m)
+//                            rounded to bf16 and written back into the same
+//                            TMEM columns (two per 32-bit column), adds p to
+//                            the row sum l
+//     O += P V_b             tcgen05.mma with A = P read from TMEM, B = V
+//                            read MN-major from its [key][d] tile, into TMEM
+//                            columns [128, 256)
+//   The running maximum m is raised only when a block's maximum exceeds it by
+//   more than 8 (in log2 units): p then stays below 2^8, and O and l, which
+//   are always relative to the same m, are rescaled by 2^(m_old - m_new) far
+//   less often than once per block.  The result is the same softmax; only
+//   the rounding differs.
+//   Two CTAs share an SM (256 TMEM columns and ~100 KB of shared memory each),
+//   so one CTA's softmax overlaps the other's MMAs.
+#pragma once
+
+#include "attn_kernel.cuh"
+
+namespace tpb {
+
+constexpr int kPrefillRows = 128;        // query rows (tokens of one head) per CTA
+constexpr int kPrefillThreads = 192;     // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
+constexpr int kPrefillTmemCols = 256;    // S / P [0, 128), O [128, 256)
+constexpr float kPrefillRescaleLog2 = 8.0f;
+
+struct PrefillParams {
+  int T;        // new tokens
+  int past;     // cached tokens before them
+  int L;        // past + T
+  int nq, G;    // query heads, query heads per key-value head
+  int ntiles;   // ceil(T / 128)
+  float scale_log2;  // log2(e) / sqrt(d)
+  uint16_t* ctx;     // [T, nq * d]
+};
+
+// Shared memory (dynamic, base rounded up to 1024 B): Q [2 d halves][128][64],
+// one K and one V stage of the same shape, barriers, the TMEM address and the
+// abort flag.
+__host__ __device__ constexpr int prefill_smem_bytes() {
+  return 1024 + 3 * kAttnBlockBytes + 10 * 8 + 16;
+}
+
+// One thread per 16-byte piece: piece fastest, then the K heads and V heads in
+// qkv's column order, then tokens, so reads of a token row are contiguous.
+__global__ void kv_append_kernel(const uint16_t* __restrict__ qkv, int T, int past, int nq,
+                                 int nkv, int max_len, uint16_t* __restrict__ k_cache,
+                                 uint16_t* __restrict__ v_cache) {
+  grid_dependency_wait();  // qkv comes from the preceding kernel
+  constexpr int kVec = kAttnHeadDim / 8;
+  const size_t per_tok = static_cast<size_t>(2) * nkv * kVec;
+  const size_t n = static_cast<size_t>(T) * per_tok;
+  const size_t ld = static_cast<size_t>(nq + 2 * nkv) * kAttnHeadDim;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t tok = e / per_tok;
+    const int rest = static_cast<int>(e - tok * per_tok);
+    const int piece = rest % kVec;
+    const int hh = (rest / kVec) % nkv;
+    const int which = rest / (kVec * nkv);  // 0 = K, 1 = V
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+        qkv + tok * ld + static_cast<size_t>(nq) * kAttnHeadDim) + rest);
+    uint16_t* cache = which ? v_cache : k_cache;
+    reinterpret_cast<uint4*>(cache + (static_cast<size_t>(hh) * max_len + past + tok) *
+                                         kAttnHeadDim)[piece] = v;
+  }
+  grid_launch_dependents();
+}
+
+__global__ void __launch_bounds__(kPrefillThreads, 2)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                        const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* qs = smem;
+  uint8_t* ks = smem + kAttnBlockBytes;
+  uint8_t* vs = smem + 2 * kAttnBlockBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * kAttnBlockBytes);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;   // S of the stage's block done
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;   // P V of the stage's block done
+  uint64_t* s_full = bars + 5;    // scores of a block in TMEM
+  uint64_t* p_full = bars + 6;    // P written (128 arrivals), O rescaled
+  uint64_t* o_done = bars + 7;    // the block's P V product done
+  uint64_t* final_bar = bars + 8; // every MMA of the issuer done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.x;                     // heads fastest: a key-value group's
+  const int tile = p.ntiles - 1 - blockIdx.y;   // heads run together; longest tiles first
+  const int q0 = tile * kPrefillRows;
+  const int g = h / p.G;
+  const int kend = p.past + q0 + kPrefillRows < p.L ? p.past + q0 + kPrefillRows : p.L;
+  const int nblk = (kend + kAttnBlockKeys - 1) / kAttnBlockKeys;  // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    mbar_init(smem_u32(k_full), 1);
+    mbar_init(smem_u32(k_empty), 1);
+    mbar_init(smem_u32(v_full), 1);
+    mbar_init(smem_u32(v_empty), 1);
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(p_full), kPrefillRows);
+    mbar_init(smem_u32(o_done), 1);
+    mbar_init(smem_u32(final_bar), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), static_cast<uint32_t>(kPrefillTmemCols));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kOCol = 128;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- TMA producer: Q once, then K_b and V_b per block, one
+      // stage each; a stage is refilled once the MMA that reads it is done
+      grid_dependency_wait();  // qkv and the appended cache rows come from preceding kernels
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      const uint32_t qb = smem_u32(q_full);
+      mbar_arrive_expect_tx(qb, kAttnBlockBytes);
+      tma_load_2d(smem_u32(qs), &tmap_q, qb, h * kAttnHeadDim, q0);
+      tma_load_2d(smem_u32(qs) + kAttnHalfBytes, &tmap_q, qb, h * kAttnHeadDim + 64, q0);
+      int kissued = 0, vissued = 0;
+      for (int b = 0; b < nblk; ++b) {
+        const int key = b * kAttnBlockKeys;
+        if (!wait_parity(smem_u32(k_empty), (b & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(smem_u32(k_full), kAttnBlockBytes);
+        tma_load_3d(smem_u32(ks), &tmap_k, smem_u32(k_full), 0, key, g);
+        tma_load_3d(smem_u32(ks) + kAttnHalfBytes, &tmap_k, smem_u32(k_full), 64, key, g);
+        ++kissued;
+        if (!wait_parity(smem_u32(v_empty), (b & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(smem_u32(v_full), kAttnBlockBytes);
+        tma_load_3d(smem_u32(vs), &tmap_v, smem_u32(v_full), 0, key, g);
+        tma_load_3d(smem_u32(vs) + kAttnHalfBytes, &tmap_v, smem_u32(v_full), 64, key, g);
+        ++vissued;
+      }
+      if (*abort_flag) {
+        // a stage is refilled only after its previous fill was consumed, so
+        // the last fill of each is the only one that can still be in flight
+        drain_wait(qb, 0, 50ull * 1000ull * 1000ull);
+        if (kissued > 0)
+          drain_wait(smem_u32(k_full), (kissued - 1) & 1, 50ull * 1000ull * 1000ull);
+        if (vissued > 0)
+          drain_wait(smem_u32(v_full), (vissued - 1) & 1, 50ull * 1000ull * 1000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- MMA issuer.  S_b overwrites the TMEM columns that hold
+      // P_{b-1}, so it waits until P_{b-1} V_{b-1} is done; the other CTA on
+      // the SM keeps the tensor core busy meanwhile.
+      const uint32_t idesc_s = idesc_bf16_f32(128, kAttnBlockKeys);              // Q, K K-major
+      const uint32_t idesc_o = idesc_bf16_f32(128, kAttnHeadDim, false, true);   // V MN-major
+      bool ok = wait_parity(smem_u32(q_full), 0, abort_flag);
+      tc_fence_after();
+      for (int b = 0; ok && b < nblk; ++b) {
+        if (b > 0 && !wait_parity(smem_u32(o_done), (b - 1) & 1, abort_flag)) break;
+        if (!wait_parity(smem_u32(k_full), b & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
+          const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
+                               static_cast<uint32_t>(kk & 3) * 32u;
+          umma_bf16(tmem, desc_kmajor_sw128(smem_u32(qs) + off),
+                    desc_kmajor_sw128(smem_u32(ks) + off), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(smem_u32(k_empty));
+        umma_commit(smem_u32(s_full));
+        if (!wait_parity(smem_u32(p_full), b & 1, abort_flag)) break;
+        if (!wait_parity(smem_u32(v_full), b & 1, abort_flag)) break;
+        tc_fence_after();
+        // K = keys in steps of 16: P columns 8 kk .. 8 kk + 7 (two keys per
+        // column); V rows 16 kk .. 16 kk + 15 = two 1024-byte core groups
+#pragma unroll
+        for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk)
+          umma_bf16_ta(tmem + kOCol, tmem + static_cast<uint32_t>(kk * 8),
+                       desc_mnmajor_sw128(smem_u32(vs) + static_cast<uint32_t>(kk) * 2048u,
+                                          kAttnHalfBytes),
+                       idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(smem_u32(v_empty));
+        umma_commit(smem_u32(o_done));
+      }
+      umma_commit(smem_u32(final_bar));
+      drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- warps 0-3: thread r owns query row r (TMEM lane r).
+    // Every thread takes the same arrivals whatever its waits returned.
+    grid_dependency_wait();  // ctx may still be read by a preceding kernel
+    const int r = threadIdx.x;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const int pos = p.past + q0 + r;  // rows at or past T are padding, never stored
+    const float c = p.scale_log2;
+    float m_used = neg_inf();
+    float l = 0.0f;
+    bool ok = true;
+    for (int b = 0; b < nblk; ++b) {
+      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(s_full), b & 1, abort_flag));
+      tc_fence_after();
+      uint32_t s[kAttnBlockKeys];
+      if (ok) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(32 * q),
+                    *reinterpret_cast<uint32_t(*)[32]>(s + 32 * q));
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int k = 0; k < kAttnBlockKeys; ++k) s[k] = 0u;
+      }
+      const int key0 = b * kAttnBlockKeys;
+      if (key0 + kAttnBlockKeys - 1 > p.past + q0) {  // a block on the diagonal
+#pragma unroll
+        for (int k = 0; k < kAttnBlockKeys; ++k)
+          if (key0 + k > pos) s[k] = __float_as_uint(neg_inf());
+      }
+      float mx4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};  // four independent chains
+#pragma unroll
+      for (int k = 0; k < kAttnBlockKeys; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], __uint_as_float(s[k]));
+      const float mb = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;  // c > 0, so the maximum commutes with the scaling
+      const bool raise = mb > m_used + kPrefillRescaleLog2;  // also the first visible key
+      float alpha = 1.0f;
+      if (raise) {
+        alpha = m_used == neg_inf() ? 0.0f : exp2_approx(m_used - mb);
+        m_used = mb;
+      }
+      l *= alpha;
+      // P in 16-column pieces, so each piece's scores die as it is stored
+      const float neg_m = -m_used;
+      float sum0 = 0.0f, sum1 = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kAttnBlockKeys / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float p0 = exp2_approx(fmaf(__uint_as_float(s[32 * q + 2 * k]), c, neg_m));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(s[32 * q + 2 * k + 1]), c, neg_m));
+          sum0 += p0;
+          sum1 += p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        if (ok) tmem_st16(tmem + lane_addr + static_cast<uint32_t>(16 * q), pk);
+      }
+      l += sum0 + sum1;
+      if (b > 0 && ok && __any_sync(0xffffffffu, raise)) {
+        // O holds the products of blocks 0 .. b - 1 (all done: S_b was issued
+        // after P_{b-1} V_{b-1} completed); lanes that keep m use alpha = 1
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          const uint32_t a = tmem + lane_addr + kOCol + static_cast<uint32_t>(32 * q);
+          tmem_ld32(a, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(a, o);
+        }
+      }
+      if (ok) tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(o_done), (nblk - 1) & 1, abort_flag));
+    tc_fence_after();
+    if (ok) {
+      const float inv = 1.0f / l;
+      const bool valid = q0 + r < p.T;
+      uint4* dst = reinterpret_cast<uint4*>(p.ctx + static_cast<size_t>(q0 + r) * p.nq * kAttnHeadDim +
+                                            static_cast<size_t>(h) * kAttnHeadDim);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_addr + kOCol + static_cast<uint32_t>(32 * q), o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            dst[4 * q + w] = make_uint4(
+                pack_bf16x2(__uint_as_float(o[8 * w]) * inv, __uint_as_float(o[8 * w + 1]) * inv),
+                pack_bf16x2(__uint_as_float(o[8 * w + 2]) * inv, __uint_as_float(o[8 * w + 3]) * inv),
+                pack_bf16x2(__uint_as_float(o[8 * w + 4]) * inv, __uint_as_float(o[8 * w + 5]) * inv),
+                pack_bf16x2(__uint_as_float(o[8 * w + 6]) * inv, __uint_as_float(o[8 * w + 7]) * inv));
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  grid_launch_dependents();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(kPrefillTmemCols));
+  }
+}
+
+}  // namespace tpb

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "attn_kernel.cuh"
+#include "attn_prefill_kernel.cuh"
 #include "colsum_kernel.cuh"
 #include "diag_kernel.cuh"
 #include "norm_kernel.cuh"
@@ -137,6 +138,15 @@ const DeviceInfo* device_info() {
                                       tpb::kPairSmemBytes),
                  "cudaFuncSetAttribute"))
       return nullptr;
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_prefill_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    tpb::prefill_smem_bytes()),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::attn_prefill_kernel,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared),
+               "cudaFuncSetAttribute"))
+    return nullptr;
   if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_decode_kernel<16>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                "cudaFuncSetAttribute") ||
@@ -878,6 +888,83 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                                     static_cast<const float*>(p.part_ml), T, n_q_heads,
                                     n_kv_heads, p.G, p.Tq, p.n_pad, p.chunks, ctx),
                  "launch attn_combine_kernel"))
+      return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
+tp_status tp_attn_prefill(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache, int T,
+                          int past, int max_len, int n_q_heads, int n_kv_heads, int head_dim,
+                          int tp_degree, tp_bf16* ctx, tp_stream_t stream) {
+  if (qkv == nullptr || k_cache == nullptr || v_cache == nullptr || ctx == nullptr)
+    return TP_ERR_NULL;
+  if (!aligned16(qkv) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(ctx))
+    return TP_ERR_ALIGN;
+  if (T < 1 || past < 0 || n_q_heads < 1 || n_kv_heads < 1 || head_dim < 1 ||
+      n_q_heads % n_kv_heads != 0 || max_len < 1 || static_cast<long long>(past) + T > max_len ||
+      static_cast<long long>(n_kv_heads) * max_len * head_dim > (1ll << 40) ||
+      (T + tpb::kPrefillRows - 1) / tpb::kPrefillRows > 65535)
+    return TP_ERR_SHAPE;
+  if (head_dim != tpb::kAttnHeadDim) return TP_ERR_UNSUPPORTED;
+  if (tp_degree < 1 || n_q_heads % tp_degree != 0 || n_kv_heads % tp_degree != 0)
+    return TP_ERR_TP_DEGREE;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return TP_ERR_CUDA;
+  if (tpb::prefill_smem_bytes() > dev->max_smem) return TP_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int nqkv = (n_q_heads + 2 * n_kv_heads) * head_dim;
+  tpb::PrefillParams p{};
+  p.T = T;
+  p.past = past;
+  p.L = past + T;
+  p.nq = n_q_heads;
+  p.G = n_q_heads / n_kv_heads;
+  p.ntiles = (T + tpb::kPrefillRows - 1) / tpb::kPrefillRows;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(tpb::kAttnHeadDim));
+  p.ctx = ctx;
+  // Q: qkv as [T, nqkv] in 64-column x 128-row boxes; K, V: {d, keys 0 .. L - 1,
+  // key-value heads} in 128-key boxes (keys at or past L read as zeros)
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, qkv, static_cast<uint64_t>(T), static_cast<uint64_t>(nqkv),
+                 tpb::kPrefillRows) ||
+      !make_tmap_rows3(&tk, k_cache, static_cast<uint64_t>(p.L), static_cast<uint64_t>(n_kv_heads),
+                       static_cast<uint64_t>(head_dim),
+                       static_cast<uint64_t>(max_len) * head_dim, tpb::kAttnBlockKeys, 1) ||
+      !make_tmap_rows3(&tv, v_cache, static_cast<uint64_t>(p.L), static_cast<uint64_t>(n_kv_heads),
+                       static_cast<uint64_t>(head_dim),
+                       static_cast<uint64_t>(max_len) * head_dim, tpb::kAttnBlockKeys, 1))
+    return TP_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  const int nattr = launch_attrs(attr, 0);
+  // 1. the new keys and values into the caches
+  {
+    const long long pieces = static_cast<long long>(T) * n_kv_heads * 2 * (head_dim / 8);
+    long long blocks = (pieces + 255) / 256;
+    if (blocks > 16ll * dev->sms) blocks = 16ll * dev->sms;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(nattr);
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::kv_append_kernel, static_cast<const uint16_t*>(qkv),
+                                    T, past, n_q_heads, n_kv_heads, max_len,
+                                    static_cast<uint16_t*>(k_cache),
+                                    static_cast<uint16_t*>(v_cache)),
+                 "launch kv_append_kernel"))
+      return TP_ERR_CUDA;
+  }
+  // 2. grid (query heads, query tiles): heads fastest, longest tiles first
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_q_heads), static_cast<unsigned>(p.ntiles), 1);
+    cfg.blockDim = dim3(tpb::kPrefillThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(tpb::prefill_smem_bytes());
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(nattr);
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::attn_prefill_kernel, tq, tk, tv, p),
+                 "launch attn_prefill_kernel"))
       return TP_ERR_CUDA;
   }
   return TP_OK;

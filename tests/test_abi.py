@@ -202,6 +202,25 @@ def test_attn_decode_rejects_bad_arguments(lib):
         tp.TP_ERR_WORKSPACE
 
 
+def test_attn_prefill_rejects_bad_arguments(lib):
+    def call(qkv=GOOD, kc=GOOD, vc=GOOD, ctx=GOOD, T=300, past=10, max_len=512, nq=64, nkv=8,
+             d=128, t=8):
+        return lib.tp_attn_prefill(qkv, kc, vc, T, past, max_len, nq, nkv, d, t, ctx, None)
+    assert call(qkv=None) == tp.TP_ERR_NULL
+    assert call(vc=None) == tp.TP_ERR_NULL
+    assert call(ctx=None) == tp.TP_ERR_NULL
+    assert call(kc=ODD) == tp.TP_ERR_ALIGN
+    assert call(ctx=ODD) == tp.TP_ERR_ALIGN
+    assert call(T=0) == tp.TP_ERR_SHAPE
+    assert call(past=-1) == tp.TP_ERR_SHAPE
+    assert call(past=300, T=300) == tp.TP_ERR_SHAPE                    # past + T > max_len
+    assert call(nq=60) == tp.TP_ERR_SHAPE                              # nkv does not divide nq
+    assert call(T=65536 * 128, max_len=65536 * 128 + 10) == tp.TP_ERR_SHAPE  # > 65535 tiles
+    assert call(d=64) == tp.TP_ERR_UNSUPPORTED
+    assert call(t=3) == tp.TP_ERR_TP_DEGREE
+    assert call(t=16) == tp.TP_ERR_TP_DEGREE                           # 8 kv heads: t <= 8
+
+
 def test_sp_norm_rejects_bad_arguments(lib):
     def call(y=GOOD, g=GOOD, T=16, H=256, t=4, eps=1e-5, r=GOOD):
         return lib.tp_sp_add_rmsnorm(y, GOOD, g, T, H, t, eps, r, GOOD, None)

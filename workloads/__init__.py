@@ -134,7 +134,9 @@ class AttnConfig:
 
 @dataclasses.dataclass(frozen=True)
 class AttnDecodeConfig:
-    """The attention core in decode: new tokens over a per-head KV cache."""
+    """The attention core: new tokens over a per-head KV cache holding `past`
+    earlier tokens (decode: a few new tokens over a long cache; prefill: a
+    whole prompt, usually with no cache)."""
     name: str
     n_q_heads: int
     n_kv_heads: int
@@ -180,6 +182,11 @@ CONFIGS: Dict[str, object] = {
     "attn70b_decode": AttnDecodeConfig("attn70b_decode", n_q_heads=64, n_kv_heads=8,
                                        head_dim=128, past=65536, tokens=(1, 2, 4),
                                        tp_degrees=(8,)),
+    # the attention core between the 70B projections, prefill: a 4096-token
+    # prompt, causal over itself (no cached tokens)
+    "attn70b_prefill": AttnDecodeConfig("attn70b_prefill", n_q_heads=64, n_kv_heads=8,
+                                        head_dim=128, past=0, tokens=(4096,),
+                                        tp_degrees=(8,)),
     # the sequence-parallel region of the 405B-shaped block in prefill
     "sp405b": SPNormConfig("sp405b", hidden=16384, tokens=(8192,), tp_degrees=(8,)),
     # 405B-shaped MLP prefill; the oracle checks 64 seeded rows
