@@ -55,12 +55,14 @@ KERNEL_SOURCES = {
     "tiled_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh"],
     "pair_gemm_kernel": ["csrc/ptx.cuh", "csrc/tiled_kernel.cuh", "csrc/pair_kernel.cuh"],
     "attn_decode_kernel": ["csrc/ptx.cuh", "csrc/attn_kernel.cuh"],
+    "attn_prefill_kernel": ["csrc/ptx.cuh", "csrc/attn_kernel.cuh", "csrc/attn_prefill_kernel.cuh"],
     "add_rmsnorm_kernel": ["csrc/ptx.cuh", "csrc/norm_kernel.cuh"],
 }
 LAUNCH_OPTIONS = {"none": 0, "pdl": 1, "pdl+static_weights": 3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # default (timed steps, warm-up steps) per workload: about a second of timed work
 DEFAULT_STEPS = {"mlp405b": (40, 5), "attn70b": (1000, 20), "attn70b_decode": (5000, 50),
+                 "attn70b_prefill": (2000, 20),
                  "mlp70b_bwd": (100, 5),
                  "sp405b": (2000, 20),
                  "mlp70b": (2000, 50),
@@ -254,6 +256,18 @@ class Workload:
             self.weights = [(d["w_qkv"].to(device), d["w_o"].to(device))]
             nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
             self.qkv = torch.empty((self.Ts[0], nqkv), dtype=torch.bfloat16, device=device)
+        elif name == "attn70b_prefill":
+            self.t = tp_degree or cfg.tp_degrees[0]
+            self.Ts = list(tokens or cfg.tokens)
+            self.xs = {T: workloads.attn_decode_qkv(cfg, T) for T in self.Ts}
+            d = cfg.head_dim
+            self.max_len = cfg.past + max(self.Ts)
+            kc = torch.empty((cfg.n_kv_heads, self.max_len, d), dtype=torch.bfloat16, device=device)
+            self.weights = [(kc, torch.empty_like(kc))]
+            # the caches each call writes and then reads (rotated like weights)
+            self.weight_bytes = 2 * cfg.n_kv_heads * self.max_len * d * 2
+            self.hidden_in = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * d
+            self.hidden_out = cfg.n_q_heads * d
         elif name == "attn70b_decode":
             self.t = tp_degree or cfg.tp_degrees[0]
             self.Ts = list(tokens or cfg.tokens)
@@ -306,7 +320,7 @@ class Workload:
         self.outs = {T: torch.empty((T, self.hidden_out), dtype=torch.bfloat16, device=device)
                      for T in self.Ts}
         # rotate weight copies so each step reads weights evicted from L2
-        assert self.weight_bytes == workload_weight_bytes(name)
+        assert tokens or self.weight_bytes == workload_weight_bytes(name)
         # (the sequence-parallel region streams activations only, all larger than L2)
         self.rot = rotation_copies(self.weight_bytes) if rotate and name != "sp405b" else 1
         if self.rot > 1:
@@ -318,6 +332,7 @@ class Workload:
                     self.weights.append(base.clone())
         self.tokens_per_step = sum(self.Ts)
         self.launches_per_step = len(self.Ts) * {"sq4096": 1, "attn70b_decode": 3,
+                                                 "attn70b_prefill": 2,
                                                  "sp405b": 1, "mlp70b_bwd": 7}.get(name, 2)
 
     def step(self, i: int, xs=None, outs=None):
@@ -346,6 +361,10 @@ class Workload:
             elif self.name == "sp405b":
                 tp.tp_sp_add_rmsnorm(xs[T], self.res[T], w, self.t, 1e-5, r_out=self.r_out[T],
                                      n_out=outs[T])
+            elif self.name == "attn70b_prefill":
+                c = self.cfg
+                tp.tp_attn_prefill(xs[T], w[0], w[1], c.past, c.n_q_heads, c.n_kv_heads,
+                                   c.head_dim, self.t, ctx=outs[T])
             elif self.name == "attn70b_decode":
                 c = self.cfg
                 tp.tp_attn_decode(xs[T], w[0], w[1], c.past, c.n_q_heads, c.n_kv_heads,
@@ -375,7 +394,12 @@ class Workload:
 
     def step_flops(self):
         """2 T per weight element (bf16 weights: 2 bytes per element); the
-        backward pass makes five GEMMs of the layer's size per step."""
+        backward pass makes five GEMMs of the layer's size per step.  Causal
+        attention: 4 d flops (q.k and p v) per query head and visible key."""
+        if self.name == "attn70b_prefill":
+            c = self.cfg
+            return sum(4 * c.head_dim * c.n_q_heads * (T * (T + 1) // 2 + c.past * T)
+                       for T in self.Ts)
         f = 0
         for T in self.Ts:
             f += 2 * T * self.weight_bytes // 2
@@ -425,6 +449,14 @@ class _OracleRunner:
             self.xs = {T: workloads.attn_decode_qkv(cfg, T) for T in cfg.tokens}
             self.k, self.v = workloads.attn_decode_cache(cfg)
             self.n_out = cfg.n_q_heads * cfg.head_dim
+        elif name == "attn70b_prefill":
+            # 8 seeded tokens of the prompt, every query head of each (tokens
+            # are independent given the keys and values they see)
+            self.t = t or cfg.tp_degrees[0]
+            T0 = cfg.tokens[0]
+            self.qkv = workloads.attn_decode_qkv(cfg, T0)
+            self.rows = workloads.sample_rows(T0, 8)
+            self.n_out = cfg.n_q_heads * cfg.head_dim
         elif name == "sq4096":
             self.t = t or cfg.tp_degrees[0]
             self.w = workloads.proj_inputs(cfg, 1)["w"]
@@ -461,6 +493,8 @@ class _OracleRunner:
             return self.x.shape[0]
         if self.name == "sp405b":
             return self.y.shape[0]
+        if self.name == "attn70b_prefill":
+            return len(self.rows)
         if self.name == "mlp70b_bwd":
             return self.x.shape[0]
         return sum(x.shape[0] for x in self.xs.values())
@@ -476,6 +510,21 @@ class _OracleRunner:
         if self.name == "sp405b":
             # 64 seeded token rows (rows are independent); one token shard
             oracle.sp_residual_norm([oracle.to_f64(self.y)], None, self.res, self.gamma, 1)
+            return 1.0
+        if self.name == "attn70b_prefill":
+            # each sampled token i against the keys and values 0 .. i of its
+            # key-value head, for all query heads
+            c = self.cfg
+            d, nq, nkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+            G = nq // nkv
+            for i in self.rows:
+                i = int(i)
+                kv = oracle.to_f64(self.qkv[:i + 1, nq * d:])
+                q = oracle.to_f64(self.qkv[i:i + 1, :nq * d])
+                for h in range(nq):
+                    g = h // G
+                    oracle.attend_head(q[:, h * d:(h + 1) * d], kv[:, g * d:(g + 1) * d],
+                                       kv[:, (nkv + g) * d:(nkv + g + 1) * d], i)
             return 1.0
         if self.name == "attn70b_decode":
             # every new token needs the whole cache: the sample is whole calls
@@ -587,6 +636,8 @@ def workload_weight_bytes(name):
         return 2 * cfg.hidden * cfg.ffn + 4 * (cfg.hidden + cfg.ffn)
     if name == "attn70b_decode":
         return 2 * cfg.n_kv_heads * cfg.past * cfg.head_dim * 2
+    if name == "attn70b_prefill":
+        return 2 * cfg.n_kv_heads * (cfg.past + max(cfg.tokens)) * cfg.head_dim * 2
     if name == "sp405b":
         return cfg.hidden * 2
     return 2 * cfg.hidden * cfg.ffn * 2
@@ -611,6 +662,9 @@ def workload_config(name, t, options, tokens=None):
                    "split by 64q/8kv heads, O-proj 8192->8192 row-split",
         "attn70b_decode": "attention core decode, 64 query / 8 key-value heads of 128 (t=8), "
                           "65536 cached tokens, T=1,2,4 new tokens per call",
+        "attn70b_prefill": "attention core prefill, 64 query / 8 key-value heads of 128 (t=8), "
+                           "a T=4096-token prompt, causal, its keys and values appended to "
+                           "the per-head caches",
         "mlp70b_bwd": "backward pass of the Llama-3-70B-shaped MLP block H=8192 F=28672, GeLU, "
                       "t=8, T=4096 tokens: dx (fused backward shard sum), dW1, dW2, db1, db2",
         "sp405b": "sequence-parallel region of the 405B-shaped block: residual add + RMSNorm "
@@ -620,10 +674,17 @@ def workload_config(name, t, options, tokens=None):
     }[name]
     wb = workload_weight_bytes(name)
     rot = rotation_copies(wb) if name != "sp405b" else 1
-    what = "KV caches" if name == "attn70b_decode" else "weights"
+    what = "KV caches" if name in ("attn70b_decode", "attn70b_prefill") else "weights"
     if tokens:
         desc += f" (token counts overridden: {list(tokens)})"
-    if name == "sp405b":
+    if name == "attn70b_prefill":
+        T0 = cfg.tokens[0]
+        nqkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+        l2 = (f"KV caches rotated per call over {rot} copies ({rot * wb / 1e6:.0f} MB); qkv "
+              f"{T0 * nqkv * 2 / 1e6:.0f} MB read and ctx {T0 * cfg.n_q_heads * cfg.head_dim * 2 / 1e6:.0f}"
+              f" MB written per call: {(T0 * nqkv * 2 + T0 * cfg.n_q_heads * cfg.head_dim * 2 + wb) / 1e6:.0f}"
+              f" MB per call > 126 MB L2")
+    elif name == "sp405b":
         l2 = (f"y, residual, r, n: {cfg.tokens[0] * cfg.hidden * 2 / 1e6:.0f} MB each > 126 MB "
               f"L2, each read or written once per step")
     else:
@@ -786,7 +847,11 @@ def kernel_durations(wl, stream, reps=5):
     tp = wl.tp
     T = wl.Ts[0]
     out = {}
-    if wl.name == "mlp70b_bwd":
+    if wl.name == "attn70b_prefill":
+        # one call: the cache append (a copy of 2 nkv d values per token, about
+        # 1 % of the time) and the attention kernel
+        calls = {"attn_prefill_kernel": (lambda: wl.step(0), wl.step_flops())}
+    elif wl.name == "mlp70b_bwd":
         # one backward pass: z recompute, dz and h, dx with the shard sum, dW1,
         # dW2 (five CTA-pair GEMMs) and the two column sums, as one call
         calls = {"pair_gemm_kernel<backward>:five_gemms": (lambda: wl.step(0), wl.step_flops())}
@@ -886,7 +951,7 @@ def parse(argv=None):
                          "not a headline configuration")
     ap.add_argument("--decode-max-tokens", type=int, default=None,
                     help="token count up to which calls take the weight-streaming kernel "
-                         "(the library's default is 64)")
+                         "(the library's default is 128)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

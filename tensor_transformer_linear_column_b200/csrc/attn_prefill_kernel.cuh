@@ -45,6 +45,14 @@ constexpr int kPrefillThreads = 192;     // warps 0-3 softmax, warp 4 TMA, warp 
 constexpr int kPrefillTmemCols = 256;    // S / P [0, 128), O [128, 256)
 constexpr float kPrefillRescaleLog2 = 8.0f;
 
+// 2^x from the hardware approximation (PTX ex2.approx.ftz.f32, relative error
+// near 2^-22, far below a bf16 rounding that follows); 2^-inf = +0.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct PrefillParams {
   int T;        // new tokens
   int past;     // cached tokens before them

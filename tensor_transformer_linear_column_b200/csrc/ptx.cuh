@@ -471,14 +471,6 @@ __device__ __forceinline__ void grid_launch_dependents() {
 
 // ------------------------------------------------------------------ epilogue math
 
-// 2^x from the hardware approximation (PTX ex2.approx.ftz.f32, relative error
-// near 2^-22, far below a bf16 rounding that follows); 2^-inf = +0.
-__device__ __forceinline__ float exp2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // tanh-form GeLU in fp32; tanh from the hardware approximation (its error is
 // far below the bf16 rounding that follows).
 __device__ __forceinline__ float tanh_approx(float x) {
