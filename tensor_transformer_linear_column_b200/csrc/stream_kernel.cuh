@@ -391,9 +391,12 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
         const int end = (g + 1) * box_seg;
         bool first = true;
         for (; i < end; ++i) {
-          if (kShards || (s & 1) == me) {
-            const int a = i & (kStreamW8Slots - 1);
-            const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
+          // 8-bit weights with two k-blocks per box: two A slots of 64 columns,
+          // box i in slot i % 2 and to issuer i % 2, so each slot has one
+          // consumer; one k-block per box: four slots of 32, issuers by stage
+          if (kShards || ((kW8 && kpb == 2) ? (i & 1) : (s & 1)) == me) {
+            const int a = kpb == 2 ? (i & 1) : (i & (kStreamW8Slots - 1));
+            const uint32_t aph = static_cast<uint32_t>(kpb == 2 ? (i >> 1) : (i >> 2)) & 1u;
             if (!wait_parity(smem_u32(kW8 ? &a_full[a] : &full_bar[s]), kW8 ? aph : ph,
                              abort_flag)) {
               ok = false;
@@ -404,8 +407,8 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
             for (int c = 0; c < kpb; ++c) {
               const uint64_t db = desc0 + ((st + xoff + static_cast<uint32_t>(c) * x_bytes) >> 4);
               if constexpr (kW8) {
-                // A: the converted bf16 k-block in TMEM slot a, 8 columns per K = 16
-                const uint32_t ta = tmem_d + a_col0 + static_cast<uint32_t>(a * 32);
+                // A: the converted bf16 k-block c of slot a, 8 columns per K = 16
+                const uint32_t ta = tmem_d + a_col0 + static_cast<uint32_t>((a * kpb + c) * 32);
 #pragma unroll
                 for (int kk = 0; kk < kStreamTileK / 16; ++kk) {
                   umma_bf16_ta(d, ta + static_cast<uint32_t>(kk * 8), db + static_cast<uint64_t>(kk * 2),
@@ -457,24 +460,26 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       uint32_t ph = 0u;
       bool ok = true;
       for (int i = 0; i < nbox; ++i) {
-        const int a = i & (kStreamW8Slots - 1);
-        const uint32_t aph = static_cast<uint32_t>(i / kStreamW8Slots) & 1u;
+        const int a = kpb == 2 ? (i & 1) : (i & (kStreamW8Slots - 1));
+        const uint32_t aph = static_cast<uint32_t>(kpb == 2 ? (i >> 1) : (i >> 2)) & 1u;
         ok = ok && wait_parity(smem_u32(&full_bar[s]), ph, abort_flag);
         ok = ok && wait_parity(smem_u32(&a_empty[a]), aph ^ 1u, abort_flag);
         // the warp stores only when all its lanes' waits succeeded (the store
         // is warp-wide); every warp arrives for every box whatever happened
         if (__all_sync(0xffffffffu, ok)) {
-          const uint8_t* row = smem + s * p.stage_bytes + t * kStreamTileK;
-          uint32_t w[32];
+          for (int c = 0; c < kpb; ++c) {
+            const uint8_t* row = smem + s * p.stage_bytes + c * kStreamW8Bytes + t * kStreamTileK;
+            uint32_t w[32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
-            const uint4 lo = e4m3x8_to_bf16x8(make_uint2(q.x, q.y));
-            const uint4 hi = e4m3x8_to_bf16x8(make_uint2(q.z, q.w));
-            w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
-            w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = *reinterpret_cast<const uint4*>(row + ((q ^ sw) << 4));
+              const uint4 lo = e4m3x8_to_bf16x8(make_uint2(v.x, v.y));
+              const uint4 hi = e4m3x8_to_bf16x8(make_uint2(v.z, v.w));
+              w[8 * q + 0] = lo.x; w[8 * q + 1] = lo.y; w[8 * q + 2] = lo.z; w[8 * q + 3] = lo.w;
+              w[8 * q + 4] = hi.x; w[8 * q + 5] = hi.y; w[8 * q + 6] = hi.z; w[8 * q + 7] = hi.w;
+            }
+            tmem_st32(tmem_d + lane_addr_c + a_col0 + static_cast<uint32_t>((a * kpb + c) * 32), w);
           }
-          tmem_st32(tmem_d + lane_addr_c + a_col0 + static_cast<uint32_t>(a * 32), w);
           tmem_wait_st();
         }
         tc_fence_before();

@@ -202,12 +202,12 @@ bool make_tmap_blocks(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 // a box {64, box_rows, 1} lands as [box_rows][64] bytes, 16-byte chunk c of
 // row r stored at chunk c ^ ((r / 2) % 4).
 bool make_tmap_blocks_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                         uint32_t box_rows) {
+                         uint32_t box_rows, uint32_t blocks) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return cuda_ok(cudaErrorSymbolNotFound, "cuTensorMapEncodeTiled lookup");
   cuuint64_t dims[3] = {64, rows, cols / 64};
   cuuint64_t strides[2] = {cols, 64};
-  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t box[3] = {64, box_rows, blocks};
   cuuint32_t estr[3] = {1, 1, 1};
   const bool ok = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -326,7 +326,10 @@ tp_status plan_stream(int max_smem, const StreamGeometry& geo, bool w8, int T, i
       tpb::stream_cta_range(p, r, lo, hi);
       even = lo % 2 == 0 && hi % 2 == 0;
     }
-    p.kpb = (!w8 && even && 6 * kb_bytes <= budget) ? 2 : 1;
+    // 8-bit weights: two k-blocks per box (16 KB of codes per request) where
+    // four such stages fit; each TMA request carries a fixed cost, and 8 KB
+    // requests left the ring waiting on the copies
+    p.kpb = (even && (w8 ? 8 * kb_bytes : 6 * kb_bytes) <= budget) ? 2 : 1;
     int kbs = budget / kb_bytes;
     kbs = kbs < 3 ? 3 : kbs;
     int stages = kbs / p.kpb;
@@ -380,7 +383,7 @@ tp_status launch_stream(const DeviceInfo& dev, const StreamGeometry& geo, const 
   CUtensorMap tw, tx;
   const bool tw_ok =
       w8 ? make_tmap_blocks_u8(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
-                               static_cast<uint32_t>(tpb::kStreamTileM))
+                               static_cast<uint32_t>(tpb::kStreamTileM), static_cast<uint32_t>(p.kpb))
          : make_tmap_blocks(&tw, w, static_cast<uint64_t>(N), static_cast<uint64_t>(K),
                             static_cast<uint32_t>(tpb::kStreamTileM), static_cast<uint32_t>(p.kpb));
   if (!tw_ok) return TP_ERR_CUDA;

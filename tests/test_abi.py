@@ -321,12 +321,13 @@ def test_stream_plan_of_the_sq4096_decode_launches():
 
 def test_stream_plan_ring_depths_of_the_70b_decode():
     # 8-bit codes are converted into tensor memory, so a stage holds only the
-    # 8 KB code tile + x: a deeper ring in the same shared memory
-    for T, stages in ((1, 11), (16, 11), (64, 6)):
+    # code tiles + x; two k-blocks per box (16 KB requests) where four such
+    # stages fit the ring's budget
+    for T, stages, kpb in ((1, 5, 2), (16, 5, 2), (64, 6, 1)):
         p = tp.tp_stream_plan(T, 8192, 28672, 1, w8=True)
-        assert p["stages"] == stages and p["kblocks_per_box"] == 1
+        assert p["stages"] == stages and p["kblocks_per_box"] == kpb, (T, p)
         t_pad = (T + 15) // 16 * 16
-        assert p["stage_bytes"] == (64 + t_pad) * 64 * 2
+        assert p["stage_bytes"] == kpb * (64 + t_pad) * 64 * 2
     # bf16 up-projection at T = 1: two k-blocks per box, three boxes in flight
     p = tp.tp_stream_plan(1, 8192, 28672)
     assert p["kblocks_per_box"] == 2 and p["stages"] == 3
@@ -371,7 +372,8 @@ def test_stream_plan_invariants(w8):
                 assert p["smem_bytes"] <= max_smem
                 assert p["smem_bytes"] >= p["stages"] * p["stage_bytes"]
                 if w8:
-                    assert p["kblocks_per_box"] == 1 and p["shards_per_cta"] <= 2
+                    assert p["shards_per_cta"] <= 2
+                    assert p["kblocks_per_box"] == 1 or p["shards_per_cta"] == 1
                 # every CTA resident at once whenever some cluster shape allows it
                 if p["grid_x"] * p["cluster"] > 2 * sms:
                     assert p["cluster"] == 1 or shards > 1
