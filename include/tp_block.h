@@ -232,7 +232,7 @@ size_t tp_attn_decode_workspace_bytes(int T, int past, int n_q_heads, int n_kv_h
  * Arithmetic: bf16 q, k, v; scores, maxima and sums in fp32; the softmax
  * weights are rounded to bf16 for the weighted sum of v (fp32 accumulate) and
  * their row sum is taken from the rounded weights; the keys are processed in
- * chunks whose partial results are merged in a fixed chunk order, so the
+ * chunks whose partial results are merged in a fixed order, so the
  * result is bit-identical from run to run and does not depend on the GPU.
  *   qkv      [T, (nq + 2 nkv) d]  tp_attn_proj_forward's qkv_out   (read)
  *   k_cache  [nkv, max_len, d]    rows [0, past) hold the cached keys;

@@ -19,7 +19,7 @@
 //                         CTAs whose chunk holds rows [past, past + T) first
 //                         copy the new tokens' K and V from qkv into them;
 //   attn_combine_kernel   per (token, query head): the partials of all chunks
-//                         merged in chunk order, divided by the total sum.
+//                         merged in a fixed order, divided by the total sum.
 //
 // attn_decode_kernel, per CTA (blocks of 128 keys; a 32 KB ring stage holds
 // one block of K or of V, loaded by TMA in the order K_0, K_1, V_0, K_2, V_1, ...):
@@ -544,21 +544,26 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
-// One warp per (token i, query head h): merge the chunk partials of head h.
-// M = max_c m_c; ctx = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c, one bf16
-// rounding.  The maximum and the sum of the l_c are taken across the lanes
-// (chunk c on lane c % 32, then a fixed butterfly); the weighted sum of the
-// o_c runs over the chunks in order, four loads in flight.  Lane l owns
-// d = 4 l .. 4 l + 3.  Every order is fixed, so the result is bit-identical
-// from run to run.
-__global__ void attn_combine_kernel(const float* __restrict__ part_o,
-                                    const float* __restrict__ part_ml, int T, int nq, int nkv,
-                                    int G, int Tq, int n_pad, int chunks,
-                                    uint16_t* __restrict__ ctx) {
+// One CTA of kCombineWarps warps per (token i, query head h): merge the chunk
+// partials of head h.  M = max_c m_c; ctx = sum_c 2^(m_c - M) o_c /
+// sum_c 2^(m_c - M) l_c, one bf16 rounding.  Every warp takes M over all
+// chunks (chunk c on lane c % 32, then a fixed butterfly); warp w sums the
+// weighted o_c and l_c of chunks w, w + kCombineWarps, ... in order, lane l
+// owning d = 4 l .. 4 l + 3; warp 0 adds the warps' sums in warp order.
+// Every order is fixed, so the result is bit-identical from run to run; the
+// chunks' loads are spread over the warps, so a merge costs about two memory
+// round trips instead of one per few chunks.
+constexpr int kCombineWarps = 8;
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                        int T, int nq, int nkv, int G, int Tq, int n_pad, int chunks,
+                        uint16_t* __restrict__ ctx) {
+  __shared__ float4 red_o[kCombineWarps][32];
+  __shared__ float red_l[kCombineWarps];
   grid_dependency_wait();
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int wid = blockIdx.x;  // (token, query head)
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= T * nq) return;
   const int i = wid / nq;
   const int h = wid % nq;
   const int g = h / G;
@@ -571,30 +576,41 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   for (int c = lane; c < chunks; c += 32) M = fmaxf(M, __ldg(ml + c * ml_stride));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float L = 0.0f;
-  for (int c = lane; c < chunks; c += 32) {
-    const float m = __ldg(ml + c * ml_stride);
-    if (m != neg_inf()) L = fmaf(exp2f(m - M), __ldg(ml + c * ml_stride + 1), L);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
   const float* po = part_o + (base * n_pad + n) * kAttnHeadDim + 4 * lane;
   const size_t o_stride = static_cast<size_t>(n_pad) * kAttnHeadDim;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.0f;
 #pragma unroll 4
-  for (int c = 0; c < chunks; ++c) {
+  for (int c = warp; c < chunks; c += kCombineWarps) {
     const float m = __ldg(ml + c * ml_stride);
-    const float w = m == neg_inf() ? 0.0f : exp2f(m - M);
+    const float l = __ldg(ml + c * ml_stride + 1);
     const float4 o = __ldg(reinterpret_cast<const float4*>(po + c * o_stride));
+    const float w = m == neg_inf() ? 0.0f : exp2f(m - M);
     acc.x = fmaf(w, o.x, acc.x);
     acc.y = fmaf(w, o.y, acc.y);
     acc.z = fmaf(w, o.z, acc.z);
     acc.w = fmaf(w, o.w, acc.w);
+    L = fmaf(w, l, L);
   }
-  const float inv = 1.0f / L;
+  red_o[warp][lane] = acc;
+  if (lane == 0) red_l[warp] = L;
+  __syncthreads();
+  if (warp != 0) return;
+  float4 sum = red_o[0][lane];
+  float lsum = red_l[0];
+#pragma unroll
+  for (int w = 1; w < kCombineWarps; ++w) {
+    const float4 v = red_o[w][lane];
+    sum.x += v.x;
+    sum.y += v.y;
+    sum.z += v.z;
+    sum.w += v.w;
+    lsum += red_l[w];
+  }
+  const float inv = 1.0f / lsum;
   uint2 packed;
-  packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-  packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  packed.x = pack_bf16x2(sum.x * inv, sum.y * inv);
+  packed.y = pack_bf16x2(sum.z * inv, sum.w * inv);
   *reinterpret_cast<uint2*>(ctx + static_cast<size_t>(i) * nq * kAttnHeadDim +
                             static_cast<size_t>(h) * kAttnHeadDim + 4 * lane) = packed;
 }

@@ -877,12 +877,11 @@ tp_status tp_attn_decode(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache,
                               : cudaLaunchKernelEx(&cfg, tpb::attn_decode_kernel<32>, tq, tk, tv, p);
     if (!cuda_ok(e, "launch attn_decode_kernel")) return TP_ERR_CUDA;
   }
-  // 2. merge the chunks of every (token, query head)
+  // 2. merge the chunks of every (token, query head): one CTA each
   {
-    const int warps = T * n_q_heads;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>((warps + 7) / 8), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(T * n_q_heads), 1, 1);
+    cfg.blockDim = dim3(tpb::kCombineWarps * 32, 1, 1);
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = static_cast<unsigned>(nattr);
