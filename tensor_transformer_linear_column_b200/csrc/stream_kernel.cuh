@@ -53,12 +53,14 @@
 // (drpranayjha.com "AI Infrastructure series, Part 5", section "Reason 2":
 // decode reads 8-bit weights).  TMA brings each k-block's 8 KB of E4M3 codes
 // into the stage (64-byte swizzle, so a thread reading its own row's 64 codes
-// hits every bank once per eight lanes); the four epilogue warps, idle while
+// hits every bank once per eight lanes; two k-blocks per box, 16 KB requests,
+// where four such stages fit the ring); the four epilogue warps, idle while
 // the weights stream, convert them (exact: every E4M3 value is a bf16 value)
 // and store the bf16 tile straight into tensor memory, one row per thread, as
 // the MMA's A operand.  So per k-block shared memory carries only the codes
 // (written by TMA, read once) and x, not a bf16 tile written and read again.
-// Four TMEM A slots decouple conversion from the MMAs.  The row scale
+// TMEM A slots decouple conversion from the MMAs: four of 32 columns (one
+// k-block each), or two of 64 with two k-blocks per box.  The row scale
 // multiplies the fp32 sum before bias and activation; HBM traffic is halved.
 //
 // Threads: warps 0-3 drain TMEM (warp w may access TMEM lanes 32w..32w+31),
@@ -106,7 +108,7 @@ constexpr int kStreamRunCols = 64;  // register running sum: t_pad <= 64 when sp
 constexpr int kStreamW8Slots = 4;   // 8-bit weights: bf16 k-blocks in TMEM (A operand slots)
 
 // TMEM columns a CTA allocates: two accumulator regions of tmem_cols each,
-// and with 8-bit weights four 32-column A slots.
+// and with 8-bit weights 128 columns of A slots (four of 32, or two of 64).
 __host__ __device__ inline int stream_tmem_alloc_cols(int tmem_cols, bool w8) {
   const int need = 2 * tmem_cols + (w8 ? kStreamW8Slots * 32 : 0);
   int c = 32;
@@ -121,7 +123,8 @@ __host__ __device__ inline int stream_tmem_alloc_cols(int tmem_cols, bool w8) {
 //                               (64-byte swizzle), converted into TMEM
 //   [.., + recv_bytes)          receive buffer [csize][R][RS] fp32: sender, row, token
 //   then barriers: full[stages], empty[stages], seg_full[2], seg_empty[2], final[2], recv,
-//   a_full[4], a_empty[4] (8-bit weights: TMEM A slots), tmem slot, abort flag
+//   a_full[4], a_empty[4] (8-bit weights: TMEM A slots; two used with two
+//   k-blocks per box), tmem slot, abort flag
 // (no receive buffer when the cluster is a single CTA: it stores directly)
 //
 // Row stride RS of the receive buffer: T rounded up to 4 floats (one 16-byte
@@ -245,7 +248,8 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   const int box_seg = nbox / p.spc;  // boxes per accumulation segment
   // two TMEM regions: the two issuers' accumulators (one segment), or
   // alternate shards (several segments)
-  // (8-bit weights: then four A slots of 32 columns, one bf16 k-block each)
+  // (8-bit weights: then the A slots, 128 columns: four of one bf16 k-block
+  // each, or two of two k-blocks)
   const uint32_t a_col0 = static_cast<uint32_t>(2 * p.tmem_cols);
   const uint32_t tcols_alloc = static_cast<uint32_t>(stream_tmem_alloc_cols(p.tmem_cols, kW8));
 
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
       int i = 0;        // box index
       int s = 0;        // its stage
       uint32_t ph = 0u;  // its pass parity
-      // 8-bit weights: box i's A slot is i % 4, its pass parity (i / 4) % 2
+      // 8-bit weights: box i's A slot and its pass parity, below
       for (int g = 0; ok && g < p.spc; ++g) {
         const int region = kShards ? (g & 1) : me;
         if (kShards && g >= 2) {
@@ -447,12 +451,13 @@ __global__ void __launch_bounds__(kStreamRegThreads, kShards ? 2 : 3)
   } else {
     if constexpr (kW8) {
       // ---------------- warps 0-3, first: E4M3 -> bf16 into TMEM.  Thread t
-      // owns TMEM lane t = weight row t of the tile: it reads its row's 64
-      // codes (four 16-byte chunks; chunk c sits at chunk c ^ ((t / 2) % 4) of
-      // the row under the 64-byte swizzle), converts them and stores the 64
-      // bf16 values as 32 columns of A slot i % 4.  Every converter thread
-      // takes every box in order, whatever its waits returned, so the warps'
-      // arrivals stay matched.
+      // owns TMEM lane t = weight row t of the tile: for each k-block c of the
+      // box it reads its row's 64 codes (four 16-byte chunks; chunk q sits at
+      // chunk q ^ ((t / 2) % 4) of the row under the 64-byte swizzle),
+      // converts them and stores the 64 bf16 values as 32 columns of box i's
+      // A slot, at column offset 32 c.  Every converter thread takes every box
+      // in order, whatever its waits returned, so the warps' arrivals stay
+      // matched.
       const int t = static_cast<int>(threadIdx.x);
       const uint32_t lane_addr_c = static_cast<uint32_t>(warp * 32) << 16;
       const int sw = (t >> 1) & 3;
