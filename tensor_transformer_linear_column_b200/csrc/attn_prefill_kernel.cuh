@@ -41,7 +41,7 @@
 namespace tpb {
 
 constexpr int kPrefillRows = 128;        // query rows (tokens of one head) per CTA
-constexpr int kPrefillThreads = 192;     // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
+constexpr int kPrefillThreads = 192;     // warps 0-3 softmax (thread 0 issues the MMAs), warp 4 TMA, warp 5 TMEM
 constexpr int kPrefillTmemCols = 256;    // S / P [0, 128), O [128, 256)
 constexpr float kPrefillRescaleLog2 = 8.0f;
 
@@ -113,7 +113,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
   uint64_t* v_full = bars + 3;
   uint64_t* v_empty = bars + 4;   // P V of the stage's block done
   uint64_t* s_full = bars + 5;    // scores of a block in TMEM
-  uint64_t* p_full = bars + 6;    // P written (128 arrivals), O rescaled
   uint64_t* o_done = bars + 7;    // the block's P V product done
   uint64_t* final_bar = bars + 8; // every MMA of the issuer done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
@@ -135,7 +134,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
     mbar_init(smem_u32(v_full), 1);
     mbar_init(smem_u32(v_empty), 1);
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_full), kPrefillRows);
     mbar_init(smem_u32(o_done), 1);
     mbar_init(smem_u32(final_bar), 1);
     *abort_flag = 0;
@@ -189,45 +187,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
     }
     __syncwarp();
   } else if (warp == 5) {
-    if (lane == 0) {
-      // ---------------- MMA issuer.  S_b overwrites the TMEM columns that hold
-      // P_{b-1}, so it waits until P_{b-1} V_{b-1} is done; the other CTA on
-      // the SM keeps the tensor core busy meanwhile.
-      const uint32_t idesc_s = idesc_bf16_f32(128, kAttnBlockKeys);              // Q, K K-major
-      const uint32_t idesc_o = idesc_bf16_f32(128, kAttnHeadDim, false, true);   // V MN-major
-      bool ok = wait_parity(smem_u32(q_full), 0, abort_flag);
-      tc_fence_after();
-      for (int b = 0; ok && b < nblk; ++b) {
-        if (b > 0 && !wait_parity(smem_u32(o_done), (b - 1) & 1, abort_flag)) break;
-        if (!wait_parity(smem_u32(k_full), b & 1, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
-                               static_cast<uint32_t>(kk & 3) * 32u;
-          umma_bf16(tmem, desc_kmajor_sw128(smem_u32(qs) + off),
-                    desc_kmajor_sw128(smem_u32(ks) + off), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(smem_u32(k_empty));
-        umma_commit(smem_u32(s_full));
-        if (!wait_parity(smem_u32(p_full), b & 1, abort_flag)) break;
-        if (!wait_parity(smem_u32(v_full), b & 1, abort_flag)) break;
-        tc_fence_after();
-        // K = keys in steps of 16: P columns 8 kk .. 8 kk + 7 (two keys per
-        // column); V rows 16 kk .. 16 kk + 15 = two 1024-byte core groups
-#pragma unroll
-        for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk)
-          umma_bf16_ta(tmem + kOCol, tmem + static_cast<uint32_t>(kk * 8),
-                       desc_mnmajor_sw128(smem_u32(vs) + static_cast<uint32_t>(kk) * 2048u,
-                                          kAttnHalfBytes),
-                       idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(smem_u32(v_empty));
-        umma_commit(smem_u32(o_done));
-      }
-      umma_commit(smem_u32(final_bar));
-      drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
-    }
-    __syncwarp();
+    __syncwarp();  // allocates and frees the TMEM; the MMAs come from softmax thread 0
   } else {
     // ---------------- warps 0-3: thread r owns query row r (TMEM lane r).
     // Every thread takes the same arrivals whatever its waits returned.
@@ -239,6 +199,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
     float m_used = neg_inf();
     float l = 0.0f;
     bool ok = true;
+    // Thread 0 issues the MMAs: S_b = Q K_b^T into TMEM columns [0, 128), and
+    // after the four warps have written P_b (a named barrier, not a round
+    // trip through another warp), O += P_b V_b.  S_{b+1} overwrites P_b, so
+    // it waits until P_b V_b is done.
+    const uint32_t idesc_s = idesc_bf16_f32(128, kAttnBlockKeys);              // Q, K K-major
+    const uint32_t idesc_o = idesc_bf16_f32(128, kAttnHeadDim, false, true);   // V MN-major
+    bool issuer_ok = true;
+    auto issue_s = [&](int b) {
+      if (!issuer_ok || !wait_parity(smem_u32(k_full), b & 1, abort_flag)) {
+        issuer_ok = false;
+        return;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
+        const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
+                             static_cast<uint32_t>(kk & 3) * 32u;
+        umma_bf16(tmem, desc_kmajor_sw128(smem_u32(qs) + off), desc_kmajor_sw128(smem_u32(ks) + off),
+                  idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(smem_u32(k_empty));
+      umma_commit(smem_u32(s_full));
+    };
+    if (r == 0) {
+      issuer_ok = wait_parity(smem_u32(q_full), 0, abort_flag);
+      issue_s(0);
+    }
     for (int b = 0; b < nblk; ++b) {
       ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(s_full), b & 1, abort_flag));
       tc_fence_after();
@@ -303,7 +290,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
       }
       if (ok) tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
+      named_barrier_sync(1, kPrefillRows);  // P_b and O's rescale are in TMEM
+      if (r == 0) {
+        tc_fence_after();
+        if (issuer_ok && wait_parity(smem_u32(v_full), b & 1, abort_flag)) {
+          // K = keys in steps of 16: P columns 8 kk .. 8 kk + 7 (two keys per
+          // column); V rows 16 kk .. 16 kk + 15 = two 1024-byte core groups
+#pragma unroll
+          for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk)
+            umma_bf16_ta(tmem + kOCol, tmem + static_cast<uint32_t>(kk * 8),
+                         desc_mnmajor_sw128(smem_u32(vs) + static_cast<uint32_t>(kk) * 2048u,
+                                            kAttnHalfBytes),
+                         idesc_o, (b > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(v_empty));
+          umma_commit(smem_u32(o_done));
+        } else {
+          issuer_ok = false;
+        }
+        if (b + 1 < nblk) {
+          if (issuer_ok && !wait_parity(smem_u32(o_done), b & 1, abort_flag)) issuer_ok = false;
+          issue_s(b + 1);
+        }
+      }
+    }
+    if (r == 0) {
+      // every MMA issued must finish before the TMEM is freed
+      umma_commit(smem_u32(final_bar));
+      drain_wait(smem_u32(final_bar), 0, 50ull * 1000ull * 1000ull);
     }
     ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(o_done), (nblk - 1) & 1, abort_flag));
     tc_fence_after();
