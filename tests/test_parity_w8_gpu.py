@@ -24,7 +24,9 @@ def _w8(shape, std, seed):
 
 
 W8_COL = [(1, 64, 64), (3, 576, 320), (5, 4096, 320), (17, 128, 1088), (63, 192, 256),
-          (64, 1024, 512), (128, 256, 384), (5, 256, 20480), (3, 8192, 320), (9, 16384, 192)]
+          (64, 1024, 512), (128, 256, 384), (5, 256, 20480), (3, 8192, 320), (9, 16384, 192),
+          # two k-blocks per box with a K-split cluster (2 CTAs, and 8 above)
+          (2, 4096, 16384)]
 
 
 @pytest.mark.parametrize("T,K,N", W8_COL)
@@ -43,7 +45,9 @@ def test_w8_colpar(T, K, N, act):
 
 
 W8_ROW = [(1, 512, 64, 1), (5, 512, 320, 2), (33, 1024, 256, 4), (64, 512, 128, 8),
-          (2, 8192, 192, 2), (8, 2048, 1088, 8), (40, 1024, 256, 16), (6, 4096, 64, 16)]
+          (2, 8192, 192, 2), (8, 2048, 1088, 8), (40, 1024, 256, 16), (6, 4096, 64, 16),
+          # two k-blocks per box, clusters of 4 (2 CTAs per shard)
+          (7, 8192, 8192, 2)]
 
 
 @pytest.mark.parametrize("T,K,N,t", W8_ROW)
