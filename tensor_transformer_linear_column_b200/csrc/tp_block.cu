@@ -138,7 +138,11 @@ const DeviceInfo* device_info() {
                                       tpb::kPairSmemBytes),
                  "cudaFuncSetAttribute"))
       return nullptr;
-  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_prefill_kernel,
+  if (!cuda_ok(cudaFuncSetAttribute(tpb::attn_prefill2_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    tpb::prefill2_smem_bytes()),
+               "cudaFuncSetAttribute") ||
+      !cuda_ok(cudaFuncSetAttribute(tpb::attn_prefill_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     tpb::prefill_smem_bytes()),
                "cudaFuncSetAttribute") ||
@@ -912,7 +916,10 @@ tp_status tp_attn_prefill(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache
     return TP_ERR_TP_DEGREE;
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return TP_ERR_CUDA;
-  if (tpb::prefill_smem_bytes() > dev->max_smem) return TP_ERR_UNSUPPORTED;
+  // an even number of query heads per key-value head: two heads per CTA
+  const bool pairs = (n_q_heads / n_kv_heads) % 2 == 0;
+  if ((pairs ? tpb::prefill2_smem_bytes() : tpb::prefill_smem_bytes()) > dev->max_smem)
+    return TP_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int nqkv = (n_q_heads + 2 * n_kv_heads) * head_dim;
   tpb::PrefillParams p{};
@@ -956,18 +963,21 @@ tp_status tp_attn_prefill(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache
                  "launch kv_append_kernel"))
       return TP_ERR_CUDA;
   }
-  // 2. grid (query heads, query tiles): heads fastest, longest tiles first
+  // 2. grid (query heads or head pairs, query tiles): heads fastest, longest
+  // tiles first
   {
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(n_q_heads), static_cast<unsigned>(p.ntiles), 1);
-    cfg.blockDim = dim3(tpb::kPrefillThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(tpb::prefill_smem_bytes());
+    cfg.gridDim = dim3(static_cast<unsigned>(pairs ? n_q_heads / 2 : n_q_heads),
+                       static_cast<unsigned>(p.ntiles), 1);
+    cfg.blockDim = dim3(pairs ? tpb::kPrefill2Threads : tpb::kPrefillThreads, 1, 1);
+    cfg.dynamicSmemBytes =
+        static_cast<size_t>(pairs ? tpb::prefill2_smem_bytes() : tpb::prefill_smem_bytes());
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = static_cast<unsigned>(nattr);
-    if (!cuda_ok(cudaLaunchKernelEx(&cfg, tpb::attn_prefill_kernel, tq, tk, tv, p),
-                 "launch attn_prefill_kernel"))
-      return TP_ERR_CUDA;
+    const cudaError_t e = pairs ? cudaLaunchKernelEx(&cfg, tpb::attn_prefill2_kernel, tq, tk, tv, p)
+                                : cudaLaunchKernelEx(&cfg, tpb::attn_prefill_kernel, tq, tk, tv, p);
+    if (!cuda_ok(e, "launch attn_prefill_kernel")) return TP_ERR_CUDA;
   }
   return TP_OK;
 }
