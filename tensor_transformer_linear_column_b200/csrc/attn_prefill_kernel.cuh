@@ -353,30 +353,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 2)
 
 // ---------------------------------------------------------------------------
 // attn_prefill2_kernel: the same operation for an even number G of query heads
-// per key-value head, two query tiles per CTA (heads h0 and h0 + 1 of one
-// key-value group, the same 128 tokens), one CTA per SM.  The tiles share
-// every K and V block.  P goes to shared memory (a K-major A operand of the
-// P V MMA) instead of back into the score columns, so a tile's softmax gives
-// its score slot back as soon as it has loaded the scores: the MMA warp then
-// computes the next block's scores while the softmax runs, and neither the
-// score MMA nor the P V MMA sits on the softmax's chain.
+// per key-value head.  A work item is two query tiles (heads h0 and h0 + 1 of
+// one key-value group, the same 128 tokens), which share every K and V block.
+// The grid is persistent, one CTA per SM: CTA c takes the items of its
+// column of a boustrophedon order over the list sorted longest first (c,
+// 2 C - 1 - c, 2 C + c, ...), so the CTAs' total key blocks agree to a few
+// per cent, and the next item's Q, K and scores are loaded while the current
+// one drains.  P goes to shared memory (a K-major A operand of the P V MMA)
+// instead of back into the score columns, so a tile's softmax gives its
+// score slot back as soon as it has loaded the scores: the MMA warp then
+// computes the next block's scores while the softmax runs.
 //   TMEM (512 columns): tile t's S at 256 t, its O at 256 t + 128.
 //   Shared memory: Q_0, Q_1, a ring of three 32 KB stages, P_0, P_1 (32 KB
 //   each: [2 halves of 64][128 rows][64] bf16, 128-byte swizzle).  The ring
-//   carries K_0, K_1, V_0, K_2, V_1, K_3, V_2, ... in the order the MMA
-//   warp reads them, so K_{b+1} is loaded once P_{b-2} V_{b-2} is done and
-//   V_b once S_b is done: both well before they are needed.
+//   carries, per item, K_0, K_1, V_0, K_2, V_1, K_3, V_2, ... in the order
+//   the MMA warp reads them, so K_{b+1} is loaded once P_{b-2} V_{b-2} is
+//   done and V_b once S_b is done: both well before they are needed.
+//   Barrier phases run on across items: the ring by its item count, the
+//   per-tile score / P / product barriers by a running block count, the Q
+//   and O-release barriers by the item count.
 //   Warps: 0-3 softmax of tile 0, 4-7 of tile 1 (thread r of a tile owns
 //   query row r), 8 TMA, 9 MMA and TMEM allocation.
 constexpr int kPrefill2Threads = 320;
 constexpr int kPrefill2Stages = 3;
 
 __host__ __device__ constexpr int prefill2_smem_bytes() {
-  return 1024 + (2 + kPrefill2Stages + 2) * kAttnBlockBytes + 20 * 8 + 16;
+  return 1024 + (2 + kPrefill2Stages + 2) * kAttnBlockBytes + 24 * 8 + 16;
 }
 
-// Ring item i (of 2 nblk): K_0, then K_{b+1} and V_b for b = 0 .. nblk - 2,
-// then V_{nblk-1}.
+// Ring item i (of 2 nblk) of a work item: K_0, then K_{b+1} and V_b for
+// b = 0 .. nblk - 2, then V_{nblk-1}.
 __device__ __forceinline__ bool ring_is_k(int i, int nblk) {
   return i == 0 || (i < 2 * nblk - 1 && ((i - 1) & 1) == 0);
 }
@@ -384,6 +390,29 @@ __device__ __forceinline__ int ring_block(int i, int nblk) {
   if (i == 0) return 0;
   if (i == 2 * nblk - 1) return nblk - 1;
   return ((i - 1) >> 1) + (((i - 1) & 1) == 0 ? 1 : 0);
+}
+
+// The r-th work item of CTA c among C (index into the longest-first list of
+// nwork items), or -1 past the end; increasing in r.
+__device__ __forceinline__ int prefill2_item(int r, int c, int C, int nwork) {
+  const int j = r * C + ((r & 1) ? (C - 1 - c) : c);
+  return j < nwork ? j : -1;
+}
+
+// Work item j: head pair j mod npairs (heads fastest, so a key-value group's
+// heads run together), tile ntiles - 1 - j / npairs (longest first).
+struct Prefill2Item {
+  int h0, q0, g, nblk;
+};
+__device__ __forceinline__ Prefill2Item prefill2_decode(int j, const PrefillParams& p) {
+  const int npairs = p.nq / 2;
+  Prefill2Item it;
+  it.h0 = (j % npairs) * 2;
+  it.q0 = (p.ntiles - 1 - j / npairs) * kPrefillRows;
+  it.g = it.h0 / p.G;  // G even: h0 and h0 + 1 share it
+  const int kend = p.past + it.q0 + kPrefillRows < p.L ? p.past + it.q0 + kPrefillRows : p.L;
+  it.nblk = (kend + kAttnBlockKeys - 1) / kAttnBlockKeys;  // >= 1
+  return it;
 }
 
 __global__ void __launch_bounds__(kPrefill2Threads, 1)
@@ -397,28 +426,27 @@ __global__ void __launch_bounds__(kPrefill2Threads, 1)
   uint8_t* ring = qs + 2 * kAttnBlockBytes;               // [kPrefill2Stages][32 KB]
   uint8_t* ps = ring + kPrefill2Stages * kAttnBlockBytes;  // [2 tiles][32 KB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2 * kAttnBlockBytes);
-  uint64_t* q_full = bars;
-  uint64_t* full = bars + 1;      // [3] per ring stage
-  uint64_t* empty = bars + 4;     // [3] both tiles' MMAs that read the stage done
-  uint64_t* s_full = bars + 7;    // [2] per tile: S of a block in TMEM
-  uint64_t* s_free = bars + 9;    // [2] per tile: the softmax has read S (128 arrivals)
-  uint64_t* p_full = bars + 11;   // [2] per tile: P in shared memory, O rescaled (128)
-  uint64_t* o_done = bars + 13;   // [2] per tile: the block's P V product done
-  uint64_t* final_bar = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars;        // an item's two Q tiles landed
+  uint64_t* q_empty = bars + 1;   // the item's last S MMAs done: Q may be replaced
+  uint64_t* full = bars + 2;      // [3] per ring stage
+  uint64_t* empty = bars + 5;     // [3] both tiles' MMAs that read the stage done
+  uint64_t* s_full = bars + 8;    // [2] per tile: S of a block in TMEM
+  uint64_t* s_free = bars + 10;   // [2] per tile: the softmax has read S (128 arrivals)
+  uint64_t* p_full = bars + 12;   // [2] per tile: P in shared memory, O rescaled (128)
+  uint64_t* o_done = bars + 14;   // [2] per tile: the block's P V product done
+  uint64_t* o_free = bars + 16;   // [2] per tile: the item's O read out (128)
+  uint64_t* final_bar = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h0 = blockIdx.x * 2;                // heads fastest, longest tiles first
-  const int tile = p.ntiles - 1 - blockIdx.y;
-  const int q0 = tile * kPrefillRows;
-  const int g = h0 / p.G;                       // G even: h0 and h0 + 1 share it
-  const int kend = p.past + q0 + kPrefillRows < p.L ? p.past + q0 + kPrefillRows : p.L;
-  const int nblk = (kend + kAttnBlockKeys - 1) / kAttnBlockKeys;  // >= 1
+  const int nwork = (p.nq / 2) * p.ntiles;
+  const int c = blockIdx.x, C = gridDim.x;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
+    mbar_init(smem_u32(q_empty), 1);
     for (int i = 0; i < kPrefill2Stages; ++i) {
       mbar_init(smem_u32(&full[i]), 1);
       mbar_init(smem_u32(&empty[i]), 1);
@@ -428,6 +456,7 @@ __global__ void __launch_bounds__(kPrefill2Threads, 1)
       mbar_init(smem_u32(&s_free[i]), kPrefillRows);
       mbar_init(smem_u32(&p_full[i]), kPrefillRows);
       mbar_init(smem_u32(&o_done[i]), 1);
+      mbar_init(smem_u32(&o_free[i]), kPrefillRows);
     }
     mbar_init(smem_u32(final_bar), 1);
     *abort_flag = 0;
@@ -444,42 +473,53 @@ __global__ void __launch_bounds__(kPrefill2Threads, 1)
 
   if (warp == 8) {
     if (lane == 0) {
-      // ---------------- TMA producer: both Q tiles, then the ring in the MMA
-      // warp's order: K_0, then per block b K_{b+1} (if any) and V_b
+      // ---------------- TMA producer: per item, both Q tiles (once the last
+      // item's last S is done), then its ring items
       grid_dependency_wait();  // qkv and the appended cache rows come from preceding kernels
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
-      const uint32_t qb = smem_u32(q_full);
-      mbar_arrive_expect_tx(qb, 2 * kAttnBlockBytes);
-      for (int t = 0; t < 2; ++t) {
-        const uint32_t dst = smem_u32(qs + t * kAttnBlockBytes);
-        tma_load_2d(dst, &tmap_q, qb, (h0 + t) * kAttnHeadDim, q0);
-        tma_load_2d(dst + kAttnHalfBytes, &tmap_q, qb, (h0 + t) * kAttnHeadDim + 64, q0);
-      }
-      const int nitems = 2 * nblk;
-      int issued = 0;
-      for (; issued < nitems; ++issued) {
-        const int st = issued % kPrefill2Stages;
-        if (!wait_parity(smem_u32(&empty[st]), ((issued / kPrefill2Stages) & 1) ^ 1, abort_flag))
-          break;
-        const int blk = ring_block(issued, nblk);
-        const uint32_t fb = smem_u32(&full[st]);
-        const uint32_t dst = smem_u32(ring + st * kAttnBlockBytes);
-        mbar_arrive_expect_tx(fb, kAttnBlockBytes);
-        if (ring_is_k(issued, nblk)) {
-          tma_load_3d(dst, &tmap_k, fb, 0, blk * kAttnBlockKeys, g);
-          tma_load_3d(dst + kAttnHalfBytes, &tmap_k, fb, 64, blk * kAttnBlockKeys, g);
-        } else {
-          tma_load_3d(dst, &tmap_v, fb, 0, blk * kAttnBlockKeys, g);
-          tma_load_3d(dst + kAttnHalfBytes, &tmap_v, fb, 64, blk * kAttnBlockKeys, g);
+      int ri = 0;  // ring items issued
+      int nq_loads = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int j = prefill2_item(r, c, C, nwork);
+        if (j < 0) break;
+        const Prefill2Item it = prefill2_decode(j, p);
+        if (r > 0 && !wait_parity(smem_u32(q_empty), (r - 1) & 1, abort_flag)) break;
+        const uint32_t qb = smem_u32(q_full);
+        mbar_arrive_expect_tx(qb, 2 * kAttnBlockBytes);
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t dst = smem_u32(qs + t * kAttnBlockBytes);
+          tma_load_2d(dst, &tmap_q, qb, (it.h0 + t) * kAttnHeadDim, it.q0);
+          tma_load_2d(dst + kAttnHalfBytes, &tmap_q, qb, (it.h0 + t) * kAttnHeadDim + 64, it.q0);
+        }
+        ++nq_loads;
+        for (int i = 0; i < 2 * it.nblk; ++i, ++ri) {
+          const int st = ri % kPrefill2Stages;
+          if (!wait_parity(smem_u32(&empty[st]), ((ri / kPrefill2Stages) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int key = ring_block(i, it.nblk) * kAttnBlockKeys;
+          const uint32_t fb = smem_u32(&full[st]);
+          const uint32_t dst = smem_u32(ring + st * kAttnBlockBytes);
+          mbar_arrive_expect_tx(fb, kAttnBlockBytes);
+          if (ring_is_k(i, it.nblk)) {
+            tma_load_3d(dst, &tmap_k, fb, 0, key, it.g);
+            tma_load_3d(dst + kAttnHalfBytes, &tmap_k, fb, 64, key, it.g);
+          } else {
+            tma_load_3d(dst, &tmap_v, fb, 0, key, it.g);
+            tma_load_3d(dst + kAttnHalfBytes, &tmap_v, fb, 64, key, it.g);
+          }
         }
       }
       if (*abort_flag) {
-        // a stage is refilled only after its previous fill was consumed, so
-        // the last fill of each stage is the only one that can be in flight
-        drain_wait(qb, 0, 50ull * 1000ull * 1000ull);
-        for (int i = issued - kPrefill2Stages < 0 ? 0 : issued - kPrefill2Stages; i < issued; ++i)
+        // a buffer is refilled only after its previous fill was consumed, so
+        // the last fill of each is the only one that can be in flight
+        if (nq_loads > 0)
+          drain_wait(smem_u32(q_full), (nq_loads - 1) & 1, 50ull * 1000ull * 1000ull);
+        for (int i = ri - kPrefill2Stages < 0 ? 0 : ri - kPrefill2Stages; i < ri; ++i)
           drain_wait(smem_u32(&full[i % kPrefill2Stages]), (i / kPrefill2Stages) & 1,
                      50ull * 1000ull * 1000ull);
       }
@@ -492,55 +532,74 @@ __global__ void __launch_bounds__(kPrefill2Threads, 1)
       // O += P_b V_b as soon as each P_b is in shared memory.
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnBlockKeys);              // Q, K K-major
       const uint32_t idesc_o = idesc_bf16_f32(128, kAttnHeadDim, false, true);   // P K-major, V MN-major
-      bool ok = wait_parity(smem_u32(q_full), 0, abort_flag);
-      const int nitems = 2 * nblk;
-      for (int i = 0; i < nitems && ok; ++i) {
-        const int st = i % kPrefill2Stages;
-        if (!wait_parity(smem_u32(&full[st]), (i / kPrefill2Stages) & 1, abort_flag)) {
+      int ci = 0;  // ring items consumed
+      int gb0 = 0;  // running index of the item's block 0
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int j = prefill2_item(r, c, C, nwork);
+        if (j < 0) break;
+        const int nblk = prefill2_decode(j, p).nblk;
+        if (!wait_parity(smem_u32(q_full), r & 1, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t base = smem_u32(ring + st * kAttnBlockBytes);
-        const int blk = ring_block(i, nblk);
-        if (ring_is_k(i, nblk)) {
-          for (int t = 0; t < 2 && ok; ++t) {  // S_blk = Q K_blk^T
-            if (blk > 0 && !wait_parity(smem_u32(&s_free[t]), (blk - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t qbase = smem_u32(qs + t * kAttnBlockBytes);
-#pragma unroll
-            for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
-              const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
-                                   static_cast<uint32_t>(kk & 3) * 32u;
-              umma_bf16(tmem + static_cast<uint32_t>(t * 256), desc_kmajor_sw128(qbase + off),
-                        desc_kmajor_sw128(base + off), idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(smem_u32(&s_full[t]));
+        for (int i = 0; i < 2 * nblk && ok; ++i, ++ci) {
+          const int st = ci % kPrefill2Stages;
+          if (!wait_parity(smem_u32(&full[st]), (ci / kPrefill2Stages) & 1, abort_flag)) {
+            ok = false;
+            break;
           }
-        } else {
-          for (int t = 0; t < 2 && ok; ++t) {  // O += P_blk V_blk
-            if (!wait_parity(smem_u32(&p_full[t]), blk & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t pbase = smem_u32(ps + t * kAttnBlockBytes);
-            // K = keys in steps of 16: P in the layout of Q (K-major, 128-byte
-            // swizzle); V rows 16 kk .. 16 kk + 15 = two 1024-byte core groups
+          const uint32_t base = smem_u32(ring + st * kAttnBlockBytes);
+          const int blk = ring_block(i, nblk);
+          const int gblk = gb0 + blk;
+          if (ring_is_k(i, nblk)) {
+            for (int t = 0; t < 2 && ok; ++t) {  // S_blk = Q K_blk^T
+              if (gblk > 0 && !wait_parity(smem_u32(&s_free[t]), (gblk - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t qbase = smem_u32(qs + t * kAttnBlockBytes);
 #pragma unroll
-            for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk) {
-              const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
-                                   static_cast<uint32_t>(kk & 3) * 32u;
-              umma_bf16(tmem + static_cast<uint32_t>(t * 256 + 128), desc_kmajor_sw128(pbase + off),
-                        desc_mnmajor_sw128(base + static_cast<uint32_t>(kk) * 2048u, kAttnHalfBytes),
-                        idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kAttnHeadDim / 16; ++kk) {
+                const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
+                                     static_cast<uint32_t>(kk & 3) * 32u;
+                umma_bf16(tmem + static_cast<uint32_t>(t * 256), desc_kmajor_sw128(qbase + off),
+                          desc_kmajor_sw128(base + off), idesc_s, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(smem_u32(&s_full[t]));
             }
-            umma_commit(smem_u32(&o_done[t]));
+            if (ok && blk == nblk - 1) umma_commit(smem_u32(q_empty));  // Q read for the last time
+          } else {
+            for (int t = 0; t < 2 && ok; ++t) {  // O += P_blk V_blk
+              if (!wait_parity(smem_u32(&p_full[t]), gblk & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              // the first product of an item overwrites O: the last item's
+              // O must have been read out
+              if (blk == 0 && r > 0 && !wait_parity(smem_u32(&o_free[t]), (r - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t pbase = smem_u32(ps + t * kAttnBlockBytes);
+              // K = keys in steps of 16: P in the layout of Q (K-major, 128-byte
+              // swizzle); V rows 16 kk .. 16 kk + 15 = two 1024-byte core groups
+#pragma unroll
+              for (int kk = 0; kk < kAttnBlockKeys / 16; ++kk) {
+                const uint32_t off = static_cast<uint32_t>(kk >> 2) * kAttnHalfBytes +
+                                     static_cast<uint32_t>(kk & 3) * 32u;
+                umma_bf16(tmem + static_cast<uint32_t>(t * 256 + 128), desc_kmajor_sw128(pbase + off),
+                          desc_mnmajor_sw128(base + static_cast<uint32_t>(kk) * 2048u, kAttnHalfBytes),
+                          idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
+              }
+              umma_commit(smem_u32(&o_done[t]));
+            }
           }
+          if (ok) umma_commit(smem_u32(&empty[st]));
         }
-        if (ok) umma_commit(smem_u32(&empty[st]));
+        gb0 += nblk;
       }
       // every MMA issued must finish before the TMEM is freed
       umma_commit(smem_u32(final_bar));
@@ -561,108 +620,118 @@ __global__ void __launch_bounds__(kPrefill2Threads, 1)
     // piece (j mod 8) xor (r mod 8) of the row's 128 bytes
     const uint32_t p_row = smem_u32(ps + t * kAttnBlockBytes) + static_cast<uint32_t>(r) * 128u;
     const uint32_t sw = static_cast<uint32_t>(r & 7);
-    const int pos = p.past + q0 + r;  // rows at or past T are padding, never stored
-    const float c = p.scale_log2;
-    float m_used = neg_inf();
-    float l = 0.0f;
+    const float c2 = p.scale_log2;
     bool ok = true;
-    for (int b = 0; b < nblk; ++b) {
-      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&s_full[t]), b & 1, abort_flag));
+    int gb0 = 0;  // running index of the item's block 0
+    for (int wi = 0;; ++wi) {
+      const int j = prefill2_item(wi, c, C, nwork);
+      if (j < 0) break;
+      const Prefill2Item it = prefill2_decode(j, p);
+      const int pos = p.past + it.q0 + r;  // rows at or past T are padding, never stored
+      float m_used = neg_inf();
+      float l = 0.0f;
+      for (int b = 0; b < it.nblk; ++b) {
+        const int gb = gb0 + b;
+        ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&s_full[t]), gb & 1, abort_flag));
+        tc_fence_after();
+        uint32_t s[kAttnBlockKeys];
+        if (ok) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tmem_ld32(s_tm + static_cast<uint32_t>(32 * q), *reinterpret_cast<uint32_t(*)[32]>(s + 32 * q));
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < kAttnBlockKeys; ++k) s[k] = 0u;
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&s_free[t]));  // the next S may overwrite the columns
+        const int key0 = b * kAttnBlockKeys;
+        if (key0 + kAttnBlockKeys - 1 > p.past + it.q0) {  // a block on the diagonal
+#pragma unroll
+          for (int k = 0; k < kAttnBlockKeys; ++k)
+            if (key0 + k > pos) s[k] = __float_as_uint(neg_inf());
+        }
+        float mx4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};  // four independent chains
+#pragma unroll
+        for (int k = 0; k < kAttnBlockKeys; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], __uint_as_float(s[k]));
+        const float mb = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c2;  // c2 > 0, so the maximum commutes with the scaling
+        const bool raise = mb > m_used + kPrefillRescaleLog2;  // also the first visible key
+        float alpha = 1.0f;
+        if (raise) {
+          alpha = m_used == neg_inf() ? 0.0f : exp2_approx(m_used - mb);
+          m_used = mb;
+        }
+        const float neg_m = -m_used;
+        float sum0 = 0.0f, sum1 = 0.0f;
+        uint32_t pk[kAttnBlockKeys / 2];
+#pragma unroll
+        for (int k = 0; k < kAttnBlockKeys / 2; ++k) {
+          const float p0 = exp2_approx(fmaf(__uint_as_float(s[2 * k]), c2, neg_m));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(s[2 * k + 1]), c2, neg_m));
+          sum0 += p0;
+          sum1 += p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + (sum0 + sum1);
+        // P replaces the previous block's P (also the last item's) and O is
+        // rescaled: both wait for the previous P V product
+        if (gb > 0)
+          ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[t]), (gb - 1) & 1, abort_flag));
+        tc_fence_after();
+#pragma unroll
+        for (int jj = 0; jj < kAttnBlockKeys / 8; ++jj) {
+          const uint32_t a = p_row + static_cast<uint32_t>(jj >> 3) * kAttnHalfBytes +
+                             ((static_cast<uint32_t>(jj & 7) ^ sw) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * jj]),
+                       "r"(pk[4 * jj + 1]), "r"(pk[4 * jj + 2]), "r"(pk[4 * jj + 3])
+                       : "memory");
+        }
+        if (b > 0 && ok && __any_sync(0xffffffffu, raise)) {
+          // lanes that keep m use alpha = 1
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            const uint32_t a = o_tm + static_cast<uint32_t>(32 * q);
+            tmem_ld32(a, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(a, o);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();  // P is read by the MMA (async proxy)
+        tc_fence_before();
+        mbar_arrive(smem_u32(&p_full[t]));
+      }
+      gb0 += it.nblk;
+      ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[t]), (gb0 - 1) & 1, abort_flag));
       tc_fence_after();
-      uint32_t s[kAttnBlockKeys];
       if (ok) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tmem_ld32(s_tm + static_cast<uint32_t>(32 * q), *reinterpret_cast<uint32_t(*)[32]>(s + 32 * q));
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int k = 0; k < kAttnBlockKeys; ++k) s[k] = 0u;
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[t]));  // S_{b+1} may overwrite the columns
-      const int key0 = b * kAttnBlockKeys;
-      if (key0 + kAttnBlockKeys - 1 > p.past + q0) {  // a block on the diagonal
-#pragma unroll
-        for (int k = 0; k < kAttnBlockKeys; ++k)
-          if (key0 + k > pos) s[k] = __float_as_uint(neg_inf());
-      }
-      float mx4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};  // four independent chains
-#pragma unroll
-      for (int k = 0; k < kAttnBlockKeys; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], __uint_as_float(s[k]));
-      const float mb = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;  // c > 0, so the maximum commutes with the scaling
-      const bool raise = mb > m_used + kPrefillRescaleLog2;  // also the first visible key
-      float alpha = 1.0f;
-      if (raise) {
-        alpha = m_used == neg_inf() ? 0.0f : exp2_approx(m_used - mb);
-        m_used = mb;
-      }
-      const float neg_m = -m_used;
-      float sum0 = 0.0f, sum1 = 0.0f;
-      uint32_t pk[kAttnBlockKeys / 2];
-#pragma unroll
-      for (int k = 0; k < kAttnBlockKeys / 2; ++k) {
-        const float p0 = exp2_approx(fmaf(__uint_as_float(s[2 * k]), c, neg_m));
-        const float p1 = exp2_approx(fmaf(__uint_as_float(s[2 * k + 1]), c, neg_m));
-        sum0 += p0;
-        sum1 += p1;
-        pk[k] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + (sum0 + sum1);
-      // P_b replaces P_{b-1} and O is rescaled: both wait for P_{b-1} V_{b-1}
-      if (b > 0)
-        ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[t]), (b - 1) & 1, abort_flag));
-      tc_fence_after();
-#pragma unroll
-      for (int j = 0; j < kAttnBlockKeys / 8; ++j) {
-        const uint32_t a = p_row + static_cast<uint32_t>(j >> 3) * kAttnHalfBytes +
-                           ((static_cast<uint32_t>(j & 7) ^ sw) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]),
-                     "r"(pk[4 * j + 1]), "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
-                     : "memory");
-      }
-      if (b > 0 && ok && __any_sync(0xffffffffu, raise)) {
-        // lanes that keep m use alpha = 1
+        const float inv = 1.0f / l;
+        const bool valid = it.q0 + r < p.T;
+        uint4* dst = reinterpret_cast<uint4*>(p.ctx + static_cast<size_t>(it.q0 + r) * p.nq * kAttnHeadDim +
+                                              static_cast<size_t>(it.h0 + t) * kAttnHeadDim);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
-          const uint32_t a = o_tm + static_cast<uint32_t>(32 * q);
-          tmem_ld32(a, o);
+          tmem_ld32(o_tm + static_cast<uint32_t>(32 * q), o);
           tmem_wait_ld();
+          if (valid) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(a, o);
+            for (int w = 0; w < 4; ++w)
+              dst[4 * q + w] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * w]) * inv, __uint_as_float(o[8 * w + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * w + 2]) * inv, __uint_as_float(o[8 * w + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * w + 4]) * inv, __uint_as_float(o[8 * w + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * w + 6]) * inv, __uint_as_float(o[8 * w + 7]) * inv));
+          }
         }
-        tmem_wait_st();
       }
-      fence_proxy_async_smem();  // P_b is read by the MMA (async proxy)
       tc_fence_before();
-      mbar_arrive(smem_u32(&p_full[t]));
+      mbar_arrive(smem_u32(&o_free[t]));  // the next item's first product may overwrite O
     }
-    ok = __all_sync(0xffffffffu, ok && wait_parity(smem_u32(&o_done[t]), (nblk - 1) & 1, abort_flag));
-    tc_fence_after();
-    if (ok) {
-      const float inv = 1.0f / l;
-      const bool valid = q0 + r < p.T;
-      uint4* dst = reinterpret_cast<uint4*>(p.ctx + static_cast<size_t>(q0 + r) * p.nq * kAttnHeadDim +
-                                            static_cast<size_t>(h0 + t) * kAttnHeadDim);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tmem_ld32(o_tm + static_cast<uint32_t>(32 * q), o);
-        tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            dst[4 * q + w] = make_uint4(
-                pack_bf16x2(__uint_as_float(o[8 * w]) * inv, __uint_as_float(o[8 * w + 1]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * w + 2]) * inv, __uint_as_float(o[8 * w + 3]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * w + 4]) * inv, __uint_as_float(o[8 * w + 5]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * w + 6]) * inv, __uint_as_float(o[8 * w + 7]) * inv));
-        }
-      }
-    }
-    tc_fence_before();
   }
   __syncthreads();
   grid_launch_dependents();

@@ -963,12 +963,14 @@ tp_status tp_attn_prefill(const tp_bf16* qkv, tp_bf16* k_cache, tp_bf16* v_cache
                  "launch kv_append_kernel"))
       return TP_ERR_CUDA;
   }
-  // 2. grid (query heads or head pairs, query tiles): heads fastest, longest
-  // tiles first
+  // 2. the attention kernel: heads fastest, longest tiles first
   {
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(pairs ? n_q_heads / 2 : n_q_heads),
-                       static_cast<unsigned>(p.ntiles), 1);
+    // two heads per CTA: a persistent grid, one CTA per SM, over (head pair,
+    // tile) items; one head per CTA: CTA (head, tile)
+    const long long items = static_cast<long long>(n_q_heads / 2) * p.ntiles;
+    cfg.gridDim = pairs ? dim3(static_cast<unsigned>(items < dev->sms ? items : dev->sms), 1, 1)
+                        : dim3(static_cast<unsigned>(n_q_heads), static_cast<unsigned>(p.ntiles), 1);
     cfg.blockDim = dim3(pairs ? tpb::kPrefill2Threads : tpb::kPrefillThreads, 1, 1);
     cfg.dynamicSmemBytes =
         static_cast<size_t>(pairs ? tpb::prefill2_smem_bytes() : tpb::prefill_smem_bytes());
