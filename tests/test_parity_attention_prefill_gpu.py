@@ -207,3 +207,37 @@ def test_attn_prefill_bench_workload_sampled_rows():
     # the caches hold every token's K and V columns
     kcols = qkv[:, nq * D:(nq + nkv) * D].reshape(T, nkv, D).transpose(0, 1)
     assert torch.equal(kd.cpu().view(torch.int16), kcols.contiguous().view(torch.int16))
+
+
+def test_attn_prefill_after_cache_many_items_per_cta_sampled_rows():
+    # 70B heads, a 2900-token chunk after 1500 cached tokens: 23 tiles x 32
+    # head pairs, about five work items per SM of different lengths, a ragged
+    # last tile; 40 seeded (token, head) rows against the oracle's one-head
+    # attention over the cached and new keys each token sees
+    dev = _dev()
+    nq, nkv, t, past, T = 64, 8, 8, 1500, 2900
+    nqkv = (nq + 2 * nkv) * D
+    qkv = workloads.random_bf16_small((T, nqkv), 1.0, 5151)
+    max_len = past + T + 7
+    kc = torch.zeros((nkv, max_len, D), dtype=torch.bfloat16)
+    vc = torch.zeros((nkv, max_len, D), dtype=torch.bfloat16)
+    kc[:, :past] = workloads.random_bf16_small((nkv, past, D), 1.0, 6151)
+    vc[:, :past] = workloads.random_bf16_small((nkv, past, D), 1.0, 7151)
+    kd, vd = kc.to(dev), vc.to(dev)
+    ctx = tp.tp_attn_prefill(qkv.to(dev), kd, vd, past, nq, nkv, D, t).cpu()
+    assert tp.tp_device_error_check() == tp.TP_OK
+    rng = np.random.default_rng(1)
+    toks = sorted(set([0, 127, 128, 2815, 2816, T - 1] + list(rng.choice(T, 34, replace=False))))
+    q64 = qkv.double().numpy()
+    kc64, vc64 = kc.double().numpy(), vc.double().numpy()
+    G = nq // nkv
+    rows, refs = [], []
+    for i in toks:
+        h = int(rng.integers(nq))
+        g = h // G
+        q = q64[i:i + 1, h * D:(h + 1) * D]
+        k = np.concatenate([kc64[g, :past], q64[:i + 1, (nq + g) * D:(nq + g + 1) * D]])
+        v = np.concatenate([vc64[g, :past], q64[:i + 1, (nq + nkv + g) * D:(nq + nkv + g + 1) * D]])
+        refs.append(oracle.attend_head(q, k, v, past + i)[0])
+        rows.append(ctx[i, h * D:(h + 1) * D])
+    _parity(torch.stack(rows), np.stack(refs), "after-cache chunk, sampled rows")

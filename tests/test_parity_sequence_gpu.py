@@ -85,3 +85,20 @@ def test_sp405b_bench_workload_sampled_rows():
     _parity(r[idx], r_ref, "sp405b r")
     _parity(n[idx], n_ref, "sp405b n")
     assert tp.tp_device_error_check() == tp.TP_OK
+
+
+@pytest.mark.parametrize("T,H,t", [(1000, 8192, 8), (450, 12288, 2), (300, 4096, 3), (149, 16384, 1)])
+def test_sp_region_wide_rows(T, H, t):
+    # wide rows kept in registers between the sum of squares and the
+    # normalisation (up to 64 values per thread), T rows in t token shards,
+    # T not a multiple of the SM count
+    dev = _dev()
+    y = workloads.random_bf16_small((T, H), 1.0, 70 + T)
+    res = workloads.random_bf16_small((T, H), 1.0, 71 + T)
+    gamma = (1.0 + workloads.random_bf16_small((H,), 0.1, 72).float()).to(torch.bfloat16)
+    r_ref, n_ref = oracle.sp_residual_norm([oracle.to_f64(y)], None, res, gamma, t)
+    r, n = tp.tp_sp_add_rmsnorm(y.to(dev), res.to(dev), gamma.to(dev), t)
+    torch.cuda.synchronize()
+    assert tp.tp_device_error_check() == tp.TP_OK
+    _parity(r, r_ref, f"r T={T} H={H}")
+    _parity(n, n_ref, f"n T={T} H={H}")
