@@ -33,7 +33,12 @@
 //   less often than once per block.  The result is the same softmax; only
 //   the rounding differs.
 //   Two CTAs share an SM (256 TMEM columns and ~100 KB of shared memory each),
-//   so one CTA's softmax overlaps the other's MMAs.
+//   so one CTA's softmax overlaps the other's MMAs.  Used for an odd number
+//   of query heads per key-value head;
+//   attn_prefill2_kernel  an even number: two heads of one key-value group
+//                         per work item, sharing every K and V block, on a
+//                         persistent grid; P goes through shared memory so
+//                         the next scores need not wait for P V (below).
 #pragma once
 
 #include "attn_kernel.cuh"
