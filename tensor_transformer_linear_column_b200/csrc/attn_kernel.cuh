@@ -546,20 +546,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
 // One CTA of kCombineWarps warps per (token i, query head h): merge the chunk
 // partials of head h.  M = max_c m_c; ctx = sum_c 2^(m_c - M) o_c /
-// sum_c 2^(m_c - M) l_c, one bf16 rounding.  Every warp takes M over all
-// chunks (chunk c on lane c % 32, then a fixed butterfly); warp w sums the
-// weighted o_c and l_c of chunks w, w + kCombineWarps, ... in order, lane l
-// owning d = 4 l .. 4 l + 3; warp 0 adds the warps' sums in warp order.
-// Every order is fixed, so the result is bit-identical from run to run; the
-// chunks' loads are spread over the warps, so a merge costs about two memory
-// round trips instead of one per few chunks.
+// sum_c 2^(m_c - M) l_c, one bf16 rounding.  Warp w takes chunks w,
+// w + kCombineWarps, ... in order with a running maximum M_w (its sums are
+// rescaled by 2^(M_w,old - M_w,new) when a chunk raises it), lane l owning
+// d = 4 l .. 4 l + 3, all of its chunks' loads issued before the first use;
+// warp 0 then takes M = max_w M_w and adds the warps' sums scaled by
+// 2^(M_w - M) in warp order.  Every order is fixed, so the result is
+// bit-identical from run to run, and a merge costs one memory round trip.
 constexpr int kCombineWarps = 8;
+constexpr int kCombineMaxPerWarp = 8;  // chunks per warp held in registers at once
 __global__ void __launch_bounds__(kCombineWarps * 32)
     attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                         int T, int nq, int nkv, int G, int Tq, int n_pad, int chunks,
                         uint16_t* __restrict__ ctx) {
   __shared__ float4 red_o[kCombineWarps][32];
   __shared__ float red_l[kCombineWarps];
+  __shared__ float red_m[kCombineWarps];
   grid_dependency_wait();
   const int wid = blockIdx.x;  // (token, query head)
   const int warp = threadIdx.x >> 5;
@@ -572,40 +574,66 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
   const size_t base = (static_cast<size_t>(grp) * nkv + g) * chunks;
   const float* ml = part_ml + (base * n_pad + n) * 2;  // chunk c at ml[c * n_pad * 2]
   const size_t ml_stride = static_cast<size_t>(n_pad) * 2;
-  float M = neg_inf();
-  for (int c = lane; c < chunks; c += 32) M = fmaxf(M, __ldg(ml + c * ml_stride));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float* po = part_o + (base * n_pad + n) * kAttnHeadDim + 4 * lane;
   const size_t o_stride = static_cast<size_t>(n_pad) * kAttnHeadDim;
+  float Mw = neg_inf();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L = 0.0f;
-#pragma unroll 4
-  for (int c = warp; c < chunks; c += kCombineWarps) {
-    const float m = __ldg(ml + c * ml_stride);
-    const float l = __ldg(ml + c * ml_stride + 1);
-    const float4 o = __ldg(reinterpret_cast<const float4*>(po + c * o_stride));
-    const float w = m == neg_inf() ? 0.0f : exp2f(m - M);
-    acc.x = fmaf(w, o.x, acc.x);
-    acc.y = fmaf(w, o.y, acc.y);
-    acc.z = fmaf(w, o.z, acc.z);
-    acc.w = fmaf(w, o.w, acc.w);
-    L = fmaf(w, l, L);
+  for (int c0 = warp; c0 < chunks; c0 += kCombineWarps * kCombineMaxPerWarp) {
+    float2 mlv[kCombineMaxPerWarp];
+    float4 ov[kCombineMaxPerWarp];
+#pragma unroll
+    for (int k = 0; k < kCombineMaxPerWarp; ++k) {
+      const int c = c0 + k * kCombineWarps;
+      if (c < chunks) {
+        mlv[k] = __ldg(reinterpret_cast<const float2*>(ml + c * ml_stride));
+        ov[k] = __ldg(reinterpret_cast<const float4*>(po + c * o_stride));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kCombineMaxPerWarp; ++k) {
+      const int c = c0 + k * kCombineWarps;
+      if (c < chunks && mlv[k].x != neg_inf()) {
+        if (mlv[k].x > Mw) {
+          const float s = Mw == neg_inf() ? 0.0f : exp2f(Mw - mlv[k].x);
+          acc.x *= s;
+          acc.y *= s;
+          acc.z *= s;
+          acc.w *= s;
+          L *= s;
+          Mw = mlv[k].x;
+        }
+        const float w = exp2f(mlv[k].x - Mw);
+        acc.x = fmaf(w, ov[k].x, acc.x);
+        acc.y = fmaf(w, ov[k].y, acc.y);
+        acc.z = fmaf(w, ov[k].z, acc.z);
+        acc.w = fmaf(w, ov[k].w, acc.w);
+        L = fmaf(w, mlv[k].y, L);
+      }
+    }
   }
   red_o[warp][lane] = acc;
-  if (lane == 0) red_l[warp] = L;
+  if (lane == 0) {
+    red_l[warp] = L;
+    red_m[warp] = Mw;
+  }
   __syncthreads();
   if (warp != 0) return;
-  float4 sum = red_o[0][lane];
-  float lsum = red_l[0];
+  float M = red_m[0];
 #pragma unroll
-  for (int w = 1; w < kCombineWarps; ++w) {
+  for (int w = 1; w < kCombineWarps; ++w) M = fmaxf(M, red_m[w]);
+  float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kCombineWarps; ++w) {
+    const float mw = red_m[w];
+    const float s = mw == neg_inf() ? 0.0f : exp2f(mw - M);
     const float4 v = red_o[w][lane];
-    sum.x += v.x;
-    sum.y += v.y;
-    sum.z += v.z;
-    sum.w += v.w;
-    lsum += red_l[w];
+    sum.x = fmaf(s, v.x, sum.x);
+    sum.y = fmaf(s, v.y, sum.y);
+    sum.z = fmaf(s, v.z, sum.z);
+    sum.w = fmaf(s, v.w, sum.w);
+    lsum = fmaf(s, red_l[w], lsum);
   }
   const float inv = 1.0f / lsum;
   uint2 packed;
