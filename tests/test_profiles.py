@@ -54,3 +54,11 @@ def test_profiles_hold_summaries_only():
     for name in os.listdir(PROFILES):
         assert name.endswith((".md", ".txt", ".json")), name
         assert os.path.getsize(os.path.join(PROFILES, name)) < 64 * 1024, name
+
+
+def test_traffic_records_match_the_current_kernel_sources():
+    # a record taken on other sources would be dropped by bench.py (traffic:
+    # null); every committed record is current
+    for key, e in _traffic().items():
+        kernel = key.rsplit(":", 1)[0]
+        assert e["source_hash"] == bench.kernel_source_hash(kernel), f"{key}: stale capture"
